@@ -1,0 +1,244 @@
+// fa_api.cu — the C ABI declared in include/fa.h: argument checks, TMA tensor
+// maps, launch configuration. No allocation per call; no host synchronisation
+// except in fa_last_device_status().
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "fa.h"
+#include "fa_fwd.cuh"
+#include "fa_bwd.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Checks shared by every tensor view of a call.
+int check_view(const fa_tensor& t, bool allow_null = false) {
+  if (t.ptr == nullptr) return allow_null ? FA_OK : FA_ERR_INVALID_ARG;
+  if (t.stride_b < 0 || t.stride_s < 0 || t.stride_h < 0) return FA_ERR_INVALID_ARG;
+  if (!aligned16(t.ptr)) return FA_ERR_MISALIGNED;
+  if ((t.stride_b % 8) || (t.stride_s % 8) || (t.stride_h % 8)) return FA_ERR_MISALIGNED;
+  return FA_OK;
+}
+
+int check_common(int B, int H, int Sq, int Sk, int D, float scale, int causal, int dtype) {
+  if (B < 1 || H < 1 || Sq < 1 || Sk < 1) return FA_ERR_INVALID_ARG;
+  if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_UNSUPPORTED;
+  if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
+  const int64_t lim = (int64_t(1) << 31) - 1;
+  if (int64_t(B) * H * Sq > lim || int64_t(B) * H * Sk > lim) return FA_ERR_INVALID_ARG;
+  if (int64_t(B) * H * ((Sq + 255) / 256) > lim) return FA_ERR_INVALID_ARG;
+  return FA_OK;
+}
+
+fa_tensor dense(const void* p, int S, int H, int D) {
+  fa_tensor t;
+  t.ptr = const_cast<void*>(p);
+  t.stride_h = D;
+  t.stride_s = int64_t(H) * D;
+  t.stride_b = int64_t(S) * H * D;
+  return t;
+}
+
+// 4-D tiled map over a [B, S, H, D] view: dims (D, S, H, B), box (64, rows, 1, 1),
+// 128-byte swizzle, out-of-range rows read as zeros.
+int make_map(CUtensorMap* map, const fa_tensor& t, int B, int S, int H, int D, int dtype, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return FA_ERR_CUDA;
+  cuuint64_t dims[4] = {cuuint64_t(D), cuuint64_t(S), cuuint64_t(H), cuuint64_t(B)};
+  cuuint64_t strides[3] = {cuuint64_t(t.stride_s) * 2, cuuint64_t(t.stride_h) * 2, cuuint64_t(t.stride_b) * 2};
+  // A stride the driver rejects (0 for an extent-1 axis) is replaced by a
+  // harmless positive one: with extent 1 it is never stepped over.
+  if (S == 1 && strides[0] == 0) strides[0] = 16;
+  if (H == 1 && strides[1] == 0) strides[1] = 16;
+  if (B == 1 && strides[2] == 0) strides[2] = 16;
+  cuuint32_t box[4] = {64, cuuint32_t(box_rows), 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, dtype == FA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4,
+                  t.ptr, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
+// Raises the dynamic shared memory limit of `fn` once per device.
+template <typename F>
+int prepare(F* fn, int smem_bytes, bool (&done)[kMaxDevices]) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
+  if (!done[dev]) {
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) != cudaSuccess)
+      return FA_ERR_CUDA;
+    done[dev] = true;
+  }
+  return FA_OK;
+}
+
+template <int D, bool BF16>
+int launch_fwd(const fa_fwd_params* p, cudaStream_t stream) {
+  using L = fa::FwdLayout<D>;
+  static bool done[kMaxDevices] = {};
+  auto* kern = &fa::fa_fwd_kernel<D, BF16>;
+  int st = prepare(kern, L::SMEM_ALLOC, done);
+  if (st != FA_OK) return st;
+  CUtensorMap mq, mk, mv;
+  if ((st = make_map(&mq, p->q, p->B, p->Sq, p->H, D, p->dtype, 128)) != FA_OK) return st;
+  if ((st = make_map(&mk, p->k, p->B, p->Sk, p->H, D, p->dtype, 128)) != FA_OK) return st;
+  if ((st = make_map(&mv, p->v, p->B, p->Sk, p->H, D, p->dtype, 128)) != FA_OK) return st;
+  fa::FwdArgs a;
+  a.o = p->o.ptr;
+  a.lse = p->lse;
+  a.o_sb = p->o.stride_b;
+  a.o_ss = p->o.stride_s;
+  a.o_sh = p->o.stride_h;
+  a.B = p->B;
+  a.H = p->H;
+  a.Sq = p->Sq;
+  a.Sk = p->Sk;
+  a.scale_log2 = p->scale * 1.4426950408889634f;
+  a.causal = p->causal;
+  a.n_qblocks = (p->Sq + 255) / 256;
+  const unsigned grid = unsigned(int64_t(a.n_qblocks) * p->B * p->H);
+  kern<<<grid, L::kThreads, L::SMEM_ALLOC, stream>>>(mq, mk, mv, a);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_version(void) { return 100; }
+
+const char* fa_strerror(int s) {
+  switch (s) {
+    case FA_OK: return "ok";
+    case FA_ERR_INVALID_ARG: return "invalid argument (null pointer, size < 1, scale or causal flag)";
+    case FA_ERR_UNSUPPORTED: return "unsupported dtype or head_dim (fp16/bf16, D in {64,128})";
+    case FA_ERR_MISALIGNED: return "tensor base or stride not 16-byte aligned";
+    case FA_ERR_CUDA: return "CUDA runtime or driver call failed";
+    case FA_ERR_TIMEOUT: return "device-side pipeline wait exceeded its time limit";
+    case FA_ERR_NOT_IMPLEMENTED: return "not implemented";
+    case FA_ERR_WORKSPACE: return "workspace missing or smaller than fa_bwd_workspace_size()";
+    default: return "unknown status";
+  }
+}
+
+int fa_fwd_ex(const fa_fwd_params* p, fa_stream_t stream) {
+  if (p == nullptr) return FA_ERR_INVALID_ARG;
+  int st = check_common(p->B, p->H, p->Sq, p->Sk, p->D, p->scale, p->causal, p->dtype);
+  if (st != FA_OK) return st;
+  const fa_tensor* views[4] = {&p->q, &p->k, &p->v, &p->o};
+  for (const fa_tensor* v : views)
+    if ((st = check_view(*v)) != FA_OK) return st;
+  if (p->lse == nullptr) return FA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(p->lse) & 3u) return FA_ERR_MISALIGNED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (p->D == 64) return p->dtype == FA_BF16 ? launch_fwd<64, true>(p, s) : launch_fwd<64, false>(p, s);
+  return p->dtype == FA_BF16 ? launch_fwd<128, true>(p, s) : launch_fwd<128, false>(p, s);
+}
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Sq, int Sk, int D,
+           float scale, int causal, int dtype, fa_stream_t stream) {
+  fa_fwd_params p;
+  std::memset(&p, 0, sizeof(p));
+  p.q = dense(q, Sq, H, D);
+  p.k = dense(k, Sk, H, D);
+  p.v = dense(v, Sk, H, D);
+  p.o = dense(o, Sq, H, D);
+  p.lse = lse;
+  p.B = B;
+  p.H = H;
+  p.Sq = Sq;
+  p.Sk = Sk;
+  p.D = D;
+  p.scale = scale;
+  p.causal = causal;
+  p.dtype = dtype;
+  return fa_fwd_ex(&p, stream);
+}
+
+size_t fa_bwd_workspace_size(int B, int H, int Sq, int D) {
+  if (B < 1 || H < 1 || Sq < 1 || D < 1) return 0;
+  const uint64_t rows = uint64_t(B) * H * ((uint64_t(Sq) + 127) / 128 * 128);
+  const uint64_t bytes = rows * uint64_t(D) * 4 + rows * 4;
+  if (bytes > (uint64_t(1) << 50)) return 0;
+  return size_t(bytes);
+}
+
+int fa_bwd_ex(const fa_bwd_params* p, fa_stream_t stream) {
+  if (p == nullptr) return FA_ERR_INVALID_ARG;
+  int st = check_common(p->B, p->H, p->Sq, p->Sk, p->D, p->scale, p->causal, p->dtype);
+  if (st != FA_OK) return st;
+  const fa_tensor* views[8] = {&p->q, &p->k, &p->v, &p->o, &p->dO, &p->dq, &p->dk, &p->dv};
+  for (const fa_tensor* v : views)
+    if ((st = check_view(*v)) != FA_OK) return st;
+  if (p->lse == nullptr) return FA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(p->lse) & 3u) return FA_ERR_MISALIGNED;
+  const size_t need = fa_bwd_workspace_size(p->B, p->H, p->Sq, p->D);
+  if (p->workspace == nullptr || p->workspace_bytes < need || need == 0) return FA_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(p->workspace) & 255u) return FA_ERR_MISALIGNED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return fa::launch_bwd(p, s);
+}
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO, void* dq,
+           void* dk, void* dv, int B, int H, int Sq, int Sk, int D, float scale, int causal, int dtype,
+           void* workspace, size_t workspace_bytes, fa_stream_t stream) {
+  fa_bwd_params p;
+  std::memset(&p, 0, sizeof(p));
+  p.q = dense(q, Sq, H, D);
+  p.k = dense(k, Sk, H, D);
+  p.v = dense(v, Sk, H, D);
+  p.o = dense(o, Sq, H, D);
+  p.dO = dense(dO, Sq, H, D);
+  p.lse = lse;
+  p.dq = dense(dq, Sq, H, D);
+  p.dk = dense(dk, Sk, H, D);
+  p.dv = dense(dv, Sk, H, D);
+  p.B = B;
+  p.H = H;
+  p.Sq = Sq;
+  p.Sk = Sk;
+  p.D = D;
+  p.scale = scale;
+  p.causal = causal;
+  p.dtype = dtype;
+  p.workspace = workspace;
+  p.workspace_bytes = workspace_bytes;
+  return fa_bwd_ex(&p, stream);
+}
+
+int fa_last_device_status(int* detail) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return FA_ERR_CUDA;
+  int h[4] = {0, 0, 0, 0};
+  if (cudaMemcpyFromSymbol(h, fa::g_status, sizeof(h)) != cudaSuccess) return FA_ERR_CUDA;
+  const int zero[4] = {0, 0, 0, 0};
+  if (cudaMemcpyToSymbol(fa::g_status, zero, sizeof(zero)) != cudaSuccess) return FA_ERR_CUDA;
+  if (detail) std::memcpy(detail, h, sizeof(h));
+  return h[0];
+}
+
+}  // extern "C"

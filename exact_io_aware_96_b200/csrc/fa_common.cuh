@@ -1,0 +1,84 @@
+// fa_common.cuh — pieces shared by the forward and backward kernels: the
+// device status word, bounded pipeline waits, and the kernel argument structs.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+
+#include "sm100.cuh"
+
+namespace fa {
+
+// Status word written by kernels whose pipeline wait ran out:
+// [0] code (FA_ERR_TIMEOUT), [1] linear block index, [2] role, [3] loop index.
+// One per device (the library is loaded once per process; every device gets
+// its own copy of a __device__ variable).
+__device__ int g_status[4];
+
+enum Role : int { kRoleLoader = 1, kRoleMma = 2, kRoleSoftmax = 3 };
+
+// A wait longer than this is treated as a hang: the kernel records it and
+// winds down instead of spinning forever. Real waits last microseconds.
+constexpr uint64_t kWaitLimitNs = 4000000000ull;
+
+__device__ __forceinline__ void record_timeout(int role, int iter) {
+  if (atomicCAS(&g_status[0], 0, -5) == 0) {
+    g_status[1] = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
+    g_status[2] = role;
+    g_status[3] = iter;
+  }
+}
+
+// Wait for phase `parity` of `bar` to complete. Returns false (and raises the
+// CTA-wide abort flag) if it has not after kWaitLimitNs, or if another warp of
+// the CTA has already aborted.
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int role,
+                                         int iter) {
+  if (sm100::mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = sm100::globaltimer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (sm100::mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (sm100::globaltimer_ns() - t0 > kWaitLimitNs) {
+      *abort_flag = 1;
+      record_timeout(role, iter);
+      return false;
+    }
+  }
+}
+
+struct FwdArgs {
+  void* o;
+  float* lse;
+  int64_t o_sb, o_ss, o_sh;  // element strides of o
+  int B, H, Sq, Sk;
+  float scale_log2;  // scale * log2(e)
+  int causal;
+  int n_qblocks;     // ceil(Sq / 256)
+};
+
+struct BwdArgs {
+  const void* o;
+  const void* dO;
+  const float* lse;
+  void* dq;
+  void* dk;
+  void* dv;
+  float* dq_acc;  // fp32 [B, H, Sq_pad, D]
+  float* dvec;    // fp32 [B, H, Sq_pad]
+  int64_t o_sb, o_ss, o_sh;
+  int64_t do_sb, do_ss, do_sh;
+  int64_t dq_sb, dq_ss, dq_sh;
+  int64_t dk_sb, dk_ss, dk_sh;
+  int64_t dv_sb, dv_ss, dv_sh;
+  int B, H, Sq, Sk, Sq_pad;
+  float scale;
+  float scale_log2;
+  int causal;
+};
+
+}  // namespace fa

@@ -1,0 +1,386 @@
+// fa_fwd.cuh — fused attention forward for sm_100a.
+//
+// One CTA computes O and LSE for 256 query rows (two 128-row tiles, t = 0, 1)
+// of one (batch, head), streaming 128-key K/V blocks through shared memory:
+// QK^T, the online softmax and PV happen in one kernel and the Sq x Sk score
+// matrix never reaches device memory ([P1] "性能引擎": fusion of the three
+// steps into one kernel; [P2] item 2 "分块处理": tiles loaded into on-chip
+// memory with an online softmax; [P5] "第三招": the next block is prefetched
+// while the current one is computed).
+//
+// Warp roles (320 threads):
+//   warps 0-3  softmax/epilogue for tile 0 (one query row per thread)
+//   warps 4-7  softmax/epilogue for tile 1
+//   warp  8    TMA loader: Q tiles once, then K_j and V_j into a ring
+//   warp  9    MMA issuer (one thread): S_t = Q_t K_j^T and O_t += P_t V_j
+// Tensor memory (512 columns x 128 lanes of fp32):
+//   [0,128) S_0   [128,256) S_1   [256,256+D) O_0   [256+D,256+2D) O_1
+//   P_t (16-bit) overwrites the first 64 columns of S_t and feeds PV as the
+//   TMEM-resident A operand.
+// Softmax per row in base 2: x = s * scale * log2(e); running max m and sum
+// l; the accumulator O_t stays unscaled and is divided by l once at the end,
+// and only LSE = ln2 * (m + log2 l) is stored ([P4] §3.1). The running max
+// is raised (and O_t, l rescaled) only when a block's max exceeds it by more
+// than 8, i.e. a factor 256; otherwise the stale max is kept, which is still
+// exact because l, O_t and LSE all use the same m.
+// Work split over batch x heads x 256-row blocks ([P4] §3.2); for causal
+// masks the grid is ordered so the longest rows start first, key blocks past
+// the diagonal are skipped and only diagonal and tail blocks are masked
+// element by element ([P4] §4: causal skips about half the blocks).
+//
+// Page legend: [P1] "Miniconda-Python3.9环境下使用FlashAttention优化训练";
+// [P2] "使用FlashAttention优化PyTorch模型注意力计算"; [P4] the FlashAttention-2
+// walkthrough titled "企业官网建设流程全解析"; [P5] the FlashAttention
+// "IO感知" overview (0539edu.com/news/165270).
+#pragma once
+
+#include "fa_common.cuh"
+
+namespace fa {
+
+template <int D>
+struct FwdLayout {
+  static constexpr int kThreads = 320;
+  static constexpr int KB = D / 64;           // 128-byte column blocks per row
+  static constexpr int TILE = 128 * D * 2;    // bytes of one 128-row tile
+  static constexpr int BLK = 128 * 128;       // bytes of one 128-row x 64-column block
+  static constexpr int STAGES = (D == 128) ? 2 : 4;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + 2 * TILE;
+  static constexpr int OFF_V = OFF_K + STAGES * TILE;
+  static constexpr int OFF_BAR = OFF_V + STAGES * TILE;
+  static constexpr int NBAR = 1 + 4 * STAGES + 2 + 2 + 2 + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int BYTES = OFF_MISC + 16;
+  static constexpr int SMEM_ALLOC = BYTES + 1024;  // room to align the base to 1024
+  static constexpr int TMEM_COLS = 512;
+};
+
+// Number of 128-key blocks that rows [r0, r0 + 128) of the query range need.
+__device__ __forceinline__ int fwd_kv_blocks(int r0, int Sq, int Sk, int causal) {
+  if (r0 >= Sq) return 0;
+  const int nk = (Sk + 127) / 128;
+  if (!causal) return nk;
+  const int last = min(r0 + 127, Sq - 1) + (Sk - Sq);
+  if (last < 0) return 0;
+  return min(nk, last / 128 + 1);
+}
+
+// Bounded wait used only on the abort path to let in-flight copies land.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = sm100::globaltimer_ns();
+  while (!sm100::mbar_try_wait(bar, parity)) {
+    if (sm100::globaltimer_ns() - t0 > 500000000ull) break;
+  }
+}
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(320, 1)
+    fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const FwdArgs a) {
+  using L = FwdLayout<D>;
+  using namespace sm100;
+  constexpr int S = L::STAGES;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+  uint64_t* q_full = bars;
+  uint64_t* k_full = bars + 1;
+  uint64_t* k_empty = k_full + S;
+  uint64_t* v_full = k_empty + S;
+  uint64_t* v_empty = v_full + S;
+  uint64_t* s_full = v_empty + S;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* o_final = p_full + 2;
+  uint64_t* drain = o_final + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // Linear block order: all heads' heaviest query blocks first (causal).
+  const int hb_count = a.H * a.B;
+  const int rank = blockIdx.x / hb_count;
+  const int hb = blockIdx.x % hb_count;
+  const int h = hb % a.H;
+  const int b = hb / a.H;
+  const int qb = a.causal ? (a.n_qblocks - 1 - rank) : rank;
+  const int q0 = qb * 256;
+  int nkv[2];
+  nkv[0] = fwd_kv_blocks(q0, a.Sq, a.Sk, a.causal);
+  nkv[1] = fwd_kv_blocks(q0 + 128, a.Sq, a.Sk, a.causal);
+  const int nmax = max(nkv[0], nkv[1]);
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&s_full[t], 1);
+      mbar_init(&p_full[t], 128);
+      mbar_init(&o_final[t], 1);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 8 && lane == 0) {
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+  }
+  if (warp == 9) {
+    tmem_alloc(tmem_slot, L::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ loader
+    if (lane == 0 && nmax > 0) {
+      int q_bytes = 0;
+      for (int t = 0; t < 2; ++t) q_bytes += nkv[t] > 0 ? L::TILE : 0;
+      mbar_arrive_expect_tx(q_full, q_bytes);
+      for (int t = 0; t < 2; ++t)
+        if (nkv[t] > 0)
+          for (int kb = 0; kb < L::KB; ++kb)
+            tma_load_4d(smem + L::OFF_Q + t * L::TILE + kb * L::BLK, &tmQ, q_full, kb * 64, q0 + 128 * t, h, b);
+      int j = 0;
+      for (; j < nmax; ++j) {
+        const int st = j % S;
+        const uint32_t ph = (j / S) & 1;
+        if (!wait_bar(&k_empty[st], ph ^ 1, abort_flag, kRoleLoader, j)) break;
+        mbar_arrive_expect_tx(&k_full[st], L::TILE);
+        for (int kb = 0; kb < L::KB; ++kb)
+          tma_load_4d(smem + L::OFF_K + st * L::TILE + kb * L::BLK, &tmK, &k_full[st], kb * 64, j * 128, h, b);
+        if (!wait_bar(&v_empty[st], ph ^ 1, abort_flag, kRoleLoader, j)) {
+          ++j;  // K_j was issued
+          break;
+        }
+        mbar_arrive_expect_tx(&v_full[st], L::TILE);
+        for (int kb = 0; kb < L::KB; ++kb)
+          tma_load_4d(smem + L::OFF_V + st * L::TILE + kb * L::BLK, &tmV, &v_full[st], kb * 64, j * 128, h, b);
+      }
+      if (*abort_flag) {
+        // Let the copies already issued land before the CTA exits.
+        drain_wait(q_full, 0);
+        for (int i = max(0, j - S); i < j; ++i) {
+          drain_wait(&k_full[i % S], (i / S) & 1);
+          drain_wait(&v_full[i % S], (i / S) & 1);
+        }
+      }
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && nmax > 0) {
+      const uint32_t idS = idesc_f16(BF16, 128, 128, 0, 0);
+      const uint32_t idO = idesc_f16(BF16, 128, D, 0, 1);
+      const uint32_t sQ = smem_u32(smem + L::OFF_Q);
+      const uint32_t sK = smem_u32(smem + L::OFF_K);
+      const uint32_t sV = smem_u32(smem + L::OFF_V);
+      auto issue_S = [&](int t, int st) {
+        const uint32_t qa = sQ + t * L::TILE;
+        const uint32_t ka = sK + st * L::TILE;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t o = (kk >> 2) * L::BLK + (kk & 3) * 32;
+          mma_ss(tmem + t * 128, desc_sw128(qa + o, 16, 1024), desc_sw128(ka + o, 16, 1024), idS, kk > 0);
+        }
+      };
+      auto issue_PV = [&](int t, int st, int acc) {
+        const uint32_t va = sV + st * L::TILE;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tmem + 256 + t * D, tmem + t * 128 + kk * 8, desc_sw128(va + kk * 2048, L::BLK, 1024), idO,
+                 (acc || kk > 0) ? 1u : 0u);
+      };
+      bool ok = wait_bar(q_full, 0, abort_flag, kRoleMma, -1) && wait_bar(&k_full[0], 0, abort_flag, kRoleMma, 0);
+      if (ok) {
+        tc_fence_after();
+        for (int t = 0; t < 2; ++t)
+          if (nkv[t] > 0) {
+            issue_S(t, 0);
+            mma_commit(&s_full[t]);
+          }
+        mma_commit(&k_empty[0]);
+      }
+      for (int j = 0; ok && j < nmax; ++j) {
+        const int st = j % S;
+        const uint32_t ph = (j / S) & 1;
+        const int jn = j + 1;
+        const int stn = jn % S;
+        const uint32_t phn = (jn / S) & 1;
+        if (!(ok = wait_bar(&v_full[st], ph, abort_flag, kRoleMma, j))) break;
+        bool kn_ready = false;
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (j < nkv[t]) {
+            if (!(ok = wait_bar(&p_full[t], j & 1, abort_flag, kRoleMma, j))) break;
+            tc_fence_after();
+            issue_PV(t, st, j > 0);
+            if (j == nkv[t] - 1) mma_commit(&o_final[t]);
+          }
+          if (jn < nkv[t]) {
+            if (!kn_ready) {
+              if (!(ok = wait_bar(&k_full[stn], phn, abort_flag, kRoleMma, jn))) break;
+              tc_fence_after();
+              kn_ready = true;
+            }
+            issue_S(t, stn);
+            mma_commit(&s_full[t]);
+          }
+        }
+        mma_commit(&v_empty[st]);
+        if (kn_ready) mma_commit(&k_empty[stn]);
+      }
+      // Wait for every MMA this thread issued before TMEM is released.
+      mma_commit(drain);
+      drain_wait(drain, 0);
+    }
+  } else {
+    // ------------------------------------------------------- softmax / epilogue
+    const int t = warp >> 2;
+    const int quarter = warp & 3;
+    const int r0 = q0 + 128 * t;
+    const int row = r0 + quarter * 32 + lane;
+    const int n = nkv[t];
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t tS = tmem + lane_base + t * 128;
+    const uint32_t tO = tmem + lane_base + 256 + t * D;
+    const float sl2 = a.scale_log2;
+    const int off = a.Sk - a.Sq;
+    float m = -INFINITY;  // running max of x = s * scale * log2(e)
+    float l = 0.f;        // running sum of 2^(x - m)
+    bool ok = true;
+
+    for (int j = 0; j < n; ++j) {
+      ok = __all_sync(0xffffffffu, wait_bar(&s_full[t], j & 1, abort_flag, kRoleSoftmax, j));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t r[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, r[c]);
+      tmem_ld_wait();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) reg_fence(r[c]);
+      float x[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int i = 0; i < 32; ++i) x[32 * c + i] = __uint_as_float(r[c][i]);
+
+      const int k0 = j * 128;
+      if (k0 + 128 > a.Sk || (a.causal && k0 + 127 > r0 + off)) {
+        int lim = a.Sk - 1 - k0;  // last allowed column of this block
+        if (a.causal) lim = min(lim, row + off - k0);
+#pragma unroll
+        for (int i = 0; i < 128; ++i) x[i] = (i <= lim) ? x[i] : -INFINITY;
+      }
+      float mx0 = x[0], mx1 = x[1], mx2 = x[2], mx3 = x[3];
+#pragma unroll
+      for (int i = 4; i < 128; i += 4) {
+        mx0 = fmaxf(mx0, x[i]);
+        mx1 = fmaxf(mx1, x[i + 1]);
+        mx2 = fmaxf(mx2, x[i + 2]);
+        mx3 = fmaxf(mx3, x[i + 3]);
+      }
+      const float m_blk = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+      const bool raise = m_blk > m + 8.0f;
+      float alpha = 1.f;
+      if (raise) {
+        alpha = ex2(m - m_blk);  // 0 when m was -inf
+        m = m_blk;
+      }
+      l *= alpha;
+      if (j > 0 && __any_sync(0xffffffffu, raise)) {
+        // Rescale this warp's 32 rows of the unscaled accumulator O_t.
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t ov[32];
+          tmem_ld32(tO + 32 * c, ov);
+          tmem_ld_wait();
+          reg_fence(ov);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+          tmem_st32(tO + 32 * c, ov);
+        }
+      }
+      const float mu = (m == -INFINITY) ? 0.f : m;
+      float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+      uint32_t p[2][32];
+#pragma unroll
+      for (int i = 0; i < 64; i += 2) {
+        const float e0 = ex2(fmaf(x[2 * i + 0], sl2, -mu));
+        const float e1 = ex2(fmaf(x[2 * i + 1], sl2, -mu));
+        const float e2 = ex2(fmaf(x[2 * i + 2], sl2, -mu));
+        const float e3 = ex2(fmaf(x[2 * i + 3], sl2, -mu));
+        s0 += e0;
+        s1 += e1;
+        s2 += e2;
+        s3 += e3;
+        p[i >> 5][i & 31] = pack2<BF16>(e0, e1);
+        p[(i + 1) >> 5][(i + 1) & 31] = pack2<BF16>(e2, e3);
+      }
+      l += (s0 + s1) + (s2 + s3);
+      tmem_st32(tS, p[0]);
+      tmem_st32(tS + 32, p[1]);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&p_full[t]);
+    }
+
+    // Epilogue: O = O_t / l, LSE = ln2 * (m + log2 l).
+    if (ok && !*abort_flag && r0 < a.Sq) {
+      const bool valid = row < a.Sq;
+      const bool has = l > 0.f;
+      const float inv_l = has ? 1.f / l : 0.f;
+      uint16_t* orow = reinterpret_cast<uint16_t*>(a.o) + static_cast<int64_t>(b) * a.o_sb +
+                       static_cast<int64_t>(row) * a.o_ss + static_cast<int64_t>(h) * a.o_sh;
+      if (n > 0) {
+        if (__all_sync(0xffffffffu, wait_bar(&o_final[t], 0, abort_flag, kRoleSoftmax, n))) {
+          tc_fence_after();
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t ov[32];
+            tmem_ld32(tO + 32 * c, ov);
+            tmem_ld_wait();
+            reg_fence(ov);
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              pk[i] = pack2<BF16>(__uint_as_float(ov[2 * i]) * inv_l, __uint_as_float(ov[2 * i + 1]) * inv_l);
+            if (valid) {
+              uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+            }
+          }
+        }
+      } else if (valid) {
+        uint4* dst = reinterpret_cast<uint4*>(orow);
+        for (int i = 0; i < D / 8; ++i) dst[i] = make_uint4(0, 0, 0, 0);
+      }
+      if (valid)
+        a.lse[(static_cast<int64_t>(b) * a.H + h) * a.Sq + row] =
+            has ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, L::TMEM_COLS);
+  }
+}
+
+}  // namespace fa

@@ -1,0 +1,197 @@
+"""ctypes binding of libfa.so: the C ABI of include/fa.h under the same names,
+plus ``forward``/``backward`` helpers that marshal torch CUDA tensors.
+
+Every computation runs in the library's kernels. There is no fallback: if
+libfa.so is missing, or a tensor is not a CUDA tensor, the call raises.
+torch is used only to allocate device memory and to name the stream.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfa.so")
+
+FA_FP16, FA_BF16 = 0, 1
+FA_OK = 0
+STATUS = {
+    0: "FA_OK", -1: "FA_ERR_INVALID_ARG", -2: "FA_ERR_UNSUPPORTED", -3: "FA_ERR_MISALIGNED",
+    -4: "FA_ERR_CUDA", -5: "FA_ERR_TIMEOUT", -6: "FA_ERR_NOT_IMPLEMENTED", -7: "FA_ERR_WORKSPACE",
+}
+EXPORTED = ("fa_fwd", "fa_fwd_ex", "fa_bwd", "fa_bwd_ex", "fa_bwd_workspace_size",
+            "fa_last_device_status", "fa_strerror", "fa_version")
+
+
+class FaTensor(ctypes.Structure):
+    _fields_ = [("ptr", ctypes.c_void_p), ("stride_b", ctypes.c_int64),
+                ("stride_s", ctypes.c_int64), ("stride_h", ctypes.c_int64)]
+
+
+class FwdParams(ctypes.Structure):
+    _fields_ = [("q", FaTensor), ("k", FaTensor), ("v", FaTensor), ("o", FaTensor),
+                ("lse", ctypes.c_void_p),
+                ("B", ctypes.c_int), ("H", ctypes.c_int), ("Sq", ctypes.c_int), ("Sk", ctypes.c_int),
+                ("D", ctypes.c_int), ("scale", ctypes.c_float), ("causal", ctypes.c_int),
+                ("dtype", ctypes.c_int)]
+
+
+class BwdParams(ctypes.Structure):
+    _fields_ = [("q", FaTensor), ("k", FaTensor), ("v", FaTensor), ("o", FaTensor), ("dO", FaTensor),
+                ("lse", ctypes.c_void_p),
+                ("dq", FaTensor), ("dk", FaTensor), ("dv", FaTensor),
+                ("B", ctypes.c_int), ("H", ctypes.c_int), ("Sq", ctypes.c_int), ("Sk", ctypes.c_int),
+                ("D", ctypes.c_int), ("scale", ctypes.c_float), ("causal", ctypes.c_int),
+                ("dtype", ctypes.c_int), ("workspace", ctypes.c_void_p),
+                ("workspace_bytes", ctypes.c_size_t)]
+
+
+class FaError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        super().__init__(f"{what}: {STATUS.get(status, status)} ({fa_strerror(status)})")
+
+
+_lib = None
+
+
+def lib():
+    """Load libfa.so (once). Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m exact_io_aware_96_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+        L.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp]
+        L.fa_fwd.restype = i
+        L.fa_fwd_ex.argtypes = [ctypes.POINTER(FwdParams), vp]
+        L.fa_fwd_ex.restype = i
+        L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp, sz, vp]
+        L.fa_bwd.restype = i
+        L.fa_bwd_ex.argtypes = [ctypes.POINTER(BwdParams), vp]
+        L.fa_bwd_ex.restype = i
+        L.fa_bwd_workspace_size.argtypes = [i, i, i, i]
+        L.fa_bwd_workspace_size.restype = sz
+        L.fa_last_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
+        L.fa_last_device_status.restype = i
+        L.fa_strerror.argtypes = [i]
+        L.fa_strerror.restype = ctypes.c_char_p
+        L.fa_version.argtypes = []
+        L.fa_version.restype = i
+        _lib = L
+    return _lib
+
+
+# ---------------------------------------------------------------- raw C ABI
+def fa_fwd(q, k, v, o, lse, B, H, Sq, Sk, D, scale, causal, dtype, stream=0) -> int:
+    return lib().fa_fwd(q, k, v, o, lse, B, H, Sq, Sk, D, scale, causal, dtype, stream)
+
+
+def fa_fwd_ex(params: FwdParams, stream=0) -> int:
+    return lib().fa_fwd_ex(ctypes.byref(params), stream)
+
+
+def fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, Sq, Sk, D, scale, causal, dtype,
+           workspace, workspace_bytes, stream=0) -> int:
+    return lib().fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, Sq, Sk, D, scale, causal, dtype,
+                        workspace, workspace_bytes, stream)
+
+
+def fa_bwd_ex(params: BwdParams, stream=0) -> int:
+    return lib().fa_bwd_ex(ctypes.byref(params), stream)
+
+
+def fa_bwd_workspace_size(B, H, Sq, D) -> int:
+    return lib().fa_bwd_workspace_size(B, H, Sq, D)
+
+
+def fa_last_device_status():
+    """(status, [code, block, role, iteration]) — synchronises the device."""
+    d = (ctypes.c_int * 4)()
+    st = lib().fa_last_device_status(d)
+    return st, list(d)
+
+
+def fa_strerror(status: int) -> str:
+    return lib().fa_strerror(status).decode()
+
+
+def fa_version() -> int:
+    return lib().fa_version()
+
+
+# ------------------------------------------------------------ torch helpers
+_DT = {torch.float16: FA_FP16, torch.bfloat16: FA_BF16}
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype not in _DT:
+        raise TypeError(f"fp16/bf16 tensors only, got {t.dtype}")
+    return _DT[t.dtype]
+
+
+def _view(t: torch.Tensor) -> FaTensor:
+    if not t.is_cuda:
+        raise ValueError("tensors must live on a CUDA device (the library has no CPU path)")
+    if t.dim() != 4 or t.stride(3) != 1:
+        raise ValueError("expected a [B, S, H, D] view with a contiguous last axis")
+    return FaTensor(t.data_ptr(), t.stride(0), t.stride(1), t.stride(2))
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def forward(q, k, v, causal=False, scale=None, out=None, lse=None, stream=None):
+    """O, LSE = attention(q, k, v) on [B, S, H, D] CUDA tensors (strided views allowed)."""
+    B, Sq, H, D = q.shape
+    Sk = k.shape[1]
+    dt = _dtype_code(q)
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError("q, k and v must share one dtype")
+    if scale is None:
+        scale = D ** -0.5
+    if out is None:
+        out = torch.empty((B, Sq, H, D), dtype=q.dtype, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, H, Sq), dtype=torch.float32, device=q.device)
+    if lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous fp32 [B, H, Sq] tensor")
+    p = FwdParams(_view(q), _view(k), _view(v), _view(out), lse.data_ptr(),
+                  B, H, Sq, Sk, D, float(scale), int(bool(causal)), dt)
+    st = fa_fwd_ex(p, _stream(stream))
+    if st != FA_OK:
+        raise FaError(st, "fa_fwd_ex")
+    return out, lse
+
+
+def workspace_for(B, H, Sq, D, device) -> torch.Tensor:
+    n = fa_bwd_workspace_size(B, H, Sq, D)
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def backward(q, k, v, o, lse, do, causal=False, scale=None, dq=None, dk=None, dv=None,
+             workspace=None, stream=None):
+    """dQ, dK, dV of L = sum(dO * O) for O = attention(q, k, v)."""
+    B, Sq, H, D = q.shape
+    Sk = k.shape[1]
+    dt = _dtype_code(q)
+    if scale is None:
+        scale = D ** -0.5
+    dq = torch.empty((B, Sq, H, D), dtype=q.dtype, device=q.device) if dq is None else dq
+    dk = torch.empty((B, Sk, H, D), dtype=q.dtype, device=q.device) if dk is None else dk
+    dv = torch.empty((B, Sk, H, D), dtype=q.dtype, device=q.device) if dv is None else dv
+    if workspace is None:
+        workspace = workspace_for(B, H, Sq, D, q.device)
+    p = BwdParams(_view(q), _view(k), _view(v), _view(o), _view(do), lse.data_ptr(),
+                  _view(dq), _view(dk), _view(dv), B, H, Sq, Sk, D, float(scale),
+                  int(bool(causal)), dt, workspace.data_ptr(), workspace.numel())
+    st = fa_bwd_ex(p, _stream(stream))
+    if st != FA_OK:
+        raise FaError(st, "fa_bwd_ex")
+    return dq, dk, dv

@@ -1,0 +1,161 @@
+/*
+ * fa.h — C ABI of the B200 (sm_100a) exact attention library, libfa.so.
+ *
+ * The library computes exact scaled dot-product attention
+ *     O = softmax(scale * Q K^T [+ causal mask]) V
+ * as one fused, tiled forward kernel that never writes the Sq x Sk score or
+ * probability matrix to device memory, and a backward that rebuilds the
+ * probabilities from the saved per-row logsumexp instead of storing them.
+ *
+ * Sources (page title, section):
+ *   [P1] "Miniconda-Python3.9环境下使用FlashAttention优化训练", section
+ *        "性能引擎：FlashAttention 如何重塑注意力计算？" (the formula; fusion of
+ *        QK^T, softmax and PV into one kernel; recomputation in the backward),
+ *        section "实战集成" (fp16/bf16 inputs; no mask or causal mask only).
+ *   [P2] "使用FlashAttention优化PyTorch模型注意力计算", section
+ *        "FlashAttention 是如何做到又快又省内存的？" items 1-3 (fusion, tiling
+ *        with an online softmax, recomputation).
+ *   [P4] the FlashAttention-2 walkthrough titled "企业官网建设流程全解析",
+ *        §3.1 (unscaled output, one final rescale, only the logsumexp saved),
+ *        §3.2 (parallelism over batch x heads x sequence blocks), §3.3 (five
+ *        matrix products in the backward), §4 (flash_attn_func on
+ *        (batch, seq_len, num_heads, head_dim), causal flag), §5 (fp32 inputs
+ *        are rejected).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Layout. q, o, dO and dq are [B, Sq, H, D]; k, v, dk and dv are [B, Sk, H, D]
+ *   (the (batch, seq_len, num_heads, head_dim) layout of [P4] §5). The
+ *   head_dim axis is contiguous. fa_fwd/fa_bwd take densely packed tensors;
+ *   the *_ex forms take per-tensor element strides for batch, sequence and
+ *   head (e.g. views into a packed qkv tensor [B, S, 3, H, D], [P1]
+ *   "实战集成").
+ * lse. fp32 [B, H, Sq], dense: LSE_i = ln sum_j exp(scale * q_i . k_j) over
+ *   the keys row i may attend to (natural log of the scaled scores; [P4] §3.1
+ *   names only "logsumexp"). A row with no allowed key gets -inf and O = 0.
+ * Causal mask. Bottom-right aligned: query i may attend to key j iff
+ *   j <= i + (Sk - Sq). With Sq == Sk this is the lower triangle.
+ * dtype. FA_FP16 or FA_BF16 for every tensor of a call except lse and the
+ *   workspace (fp32). Anything else is FA_ERR_UNSUPPORTED ([P4] §5).
+ * head_dim. D in {64, 128}; other values are FA_ERR_UNSUPPORTED.
+ * scale. Finite and > 0 (1/sqrt(D) in the usual use); else FA_ERR_INVALID_ARG.
+ * Sizes. B, H, Sq, Sk >= 1; B*H*Sq and B*H*Sk below 2^31.
+ * Alignment. Every tensor base address 16-byte aligned and every stride a
+ *   multiple of 8 elements (16 bytes): the kernels read tiles with the Tensor
+ *   Memory Accelerator. Violations are FA_ERR_MISALIGNED.
+ * Ownership. The caller allocates every tensor and the workspace, in device
+ *   memory of the current device, and owns the stream. The library keeps no
+ *   per-call allocations: it holds one device status word per device.
+ * Asynchrony. Calls enqueue work on `stream` and return without waiting.
+ *   Argument errors are detected on the host before anything is launched and
+ *   return a negative fa_status with no work enqueued. A failed launch
+ *   returns FA_ERR_CUDA. Errors detected inside a running kernel (a pipeline
+ *   wait that exceeded its time limit) are recorded in the device status word
+ *   and reported by fa_last_device_status().
+ * Streams. `stream` is a cudaStream_t (0 = the legacy default stream).
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;
+typedef struct CUstream_st* fa_stream_t; /* identical to cudaStream_t */
+
+typedef enum { FA_FP16 = 0, FA_BF16 = 1 } fa_dtype;
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = -1,     /* null pointer, size < 1, bad scale or causal flag */
+  FA_ERR_UNSUPPORTED = -2,     /* dtype or head_dim outside what the kernels handle */
+  FA_ERR_MISALIGNED = -3,      /* base address or stride breaks the 16-byte rule */
+  FA_ERR_CUDA = -4,            /* a CUDA runtime/driver call failed */
+  FA_ERR_TIMEOUT = -5,         /* a device-side pipeline wait ran out (fa_last_device_status) */
+  FA_ERR_NOT_IMPLEMENTED = -6, /* reserved */
+  FA_ERR_WORKSPACE = -7        /* workspace pointer null or smaller than fa_bwd_workspace_size */
+} fa_status;
+
+/* A strided [B, S, H, D] view: element strides for batch, sequence and head;
+   the head_dim axis has stride 1. */
+typedef struct {
+  void* ptr;
+  int64_t stride_b, stride_s, stride_h;
+} fa_tensor;
+
+typedef struct {
+  fa_tensor q, k, v; /* read */
+  fa_tensor o;       /* written */
+  float* lse;        /* written, dense fp32 [B, H, Sq] */
+  int B, H, Sq, Sk, D;
+  float scale;
+  int causal; /* 0 or 1 */
+  int dtype;  /* fa_dtype */
+} fa_fwd_params;
+
+typedef struct {
+  fa_tensor q, k, v, o, dO; /* read; o and lse are the forward's outputs */
+  const float* lse;         /* read, dense fp32 [B, H, Sq] */
+  fa_tensor dq, dk, dv;     /* written */
+  int B, H, Sq, Sk, D;
+  float scale;
+  int causal;
+  int dtype;
+  void* workspace; /* device scratch, >= fa_bwd_workspace_size(B, H, Sq, D) bytes, 256-byte aligned */
+  size_t workspace_bytes;
+} fa_bwd_params;
+
+/* Forward ([P1] "性能引擎"; [P2] items 1-2; [P4] §3.1, §3.2).
+   Reads q [B,Sq,H,D], k and v [B,Sk,H,D]; writes o [B,Sq,H,D] (rounded once,
+   to nearest even, to `dtype`) and lse [B,H,Sq] fp32. Dense tensors. */
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+           int B, int H, int Sq, int Sk, int D, float scale, int causal,
+           int dtype, fa_stream_t stream);
+
+/* Forward on strided views (packed qkv and the like). Same semantics. */
+int fa_fwd_ex(const fa_fwd_params* p, fa_stream_t stream);
+
+/* Backward ([P1] "性能引擎" recomputation; [P2] item 3; [P4] §3.1 logsumexp,
+   §3.3 five matrix products). Given the forward's inputs, its outputs o and
+   lse, and dO = dL/dO, writes dq, dk, dv = dL/dq, dL/dk, dL/dv (each rounded
+   once to `dtype`). P is rebuilt from lse, never read from memory. dq is
+   accumulated in fp32 in `workspace` and converted at the end; the
+   accumulation order across key blocks is not fixed, so dq may differ in the
+   last bits from run to run. The workspace contents on entry do not matter;
+   the call overwrites them. */
+int fa_bwd(const void* q, const void* k, const void* v, const void* o,
+           const float* lse, const void* dO, void* dq, void* dk, void* dv,
+           int B, int H, int Sq, int Sk, int D, float scale, int causal,
+           int dtype, void* workspace, size_t workspace_bytes,
+           fa_stream_t stream);
+
+/* Backward on strided views. Same semantics. */
+int fa_bwd_ex(const fa_bwd_params* p, fa_stream_t stream);
+
+/* Bytes of device workspace fa_bwd needs: an fp32 dq accumulator and the fp32
+   row terms Dvec_i = sum_d dO_id O_id, each padded to whole 128-row blocks.
+   Returns 0 for sizes < 1 or on overflow. */
+size_t fa_bwd_workspace_size(int B, int H, int Sq, int D);
+
+/* Synchronises the current device, returns the status word recorded by
+   kernels since the last call (FA_OK or FA_ERR_TIMEOUT) and clears it.
+   FA_ERR_CUDA if the device cannot be queried. If `detail` is non-null it
+   receives 4 ints: code, linear block index, role (1 = loader, 2 = MMA
+   issuer, 3 = softmax/epilogue) and the block-loop iteration. */
+int fa_last_device_status(int* detail);
+
+/* Static, human-readable text for a status code. Never null. */
+const char* fa_strerror(int status);
+
+/* Library ABI version: major * 10000 + minor * 100 + patch. */
+int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H_ */

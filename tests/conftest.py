@@ -8,3 +8,15 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200) and the built libfa.so")
+
+
+import pytest  # noqa: E402
+
+
+@pytest.fixture(scope="session")
+def fa_lib():
+    """The built libfa.so (built in-tree first if it is missing)."""
+    from exact_io_aware_96_b200 import build, fa
+    if not os.path.exists(fa.LIB_PATH):
+        build.build()
+    return fa.lib()

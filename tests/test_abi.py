@@ -1,0 +1,101 @@
+"""The C ABI without a GPU: libfa.so loads, exports what include/fa.h declares,
+and rejects bad arguments on the host (no CUDA call is reached)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from exact_io_aware_96_b200 import fa
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "fa.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(fa_\w+)\s*\(", src, flags=re.M)))
+
+
+def test_header_lists_expected_entry_points():
+    assert set(declared_functions()) == set(fa.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(fa_lib):
+    for name in declared_functions():
+        assert hasattr(fa_lib, name), name
+
+
+def test_version_and_strerror(fa_lib):
+    assert fa.fa_version() >= 100
+    for code in fa.STATUS:
+        assert fa.fa_strerror(code)
+    assert fa.fa_strerror(12345) == "unknown status"
+
+
+def test_workspace_size(fa_lib):
+    # dq accumulator (fp32, rows padded to 128) + Dvec (fp32)
+    assert fa.fa_bwd_workspace_size(1, 2, 128, 64) == 2 * 128 * 64 * 4 + 2 * 128 * 4
+    assert fa.fa_bwd_workspace_size(2, 12, 2000, 64) == 24 * 2048 * 64 * 4 + 24 * 2048 * 4
+    assert fa.fa_bwd_workspace_size(0, 1, 1, 64) == 0
+    assert fa.fa_bwd_workspace_size(1, 1, -5, 64) == 0
+
+
+A = 0x10000  # a 16-byte aligned fake address: validation fails before any use
+
+
+def fwd(**kw):
+    args = dict(q=A, k=A, v=A, o=A, lse=A, B=1, H=2, Sq=128, Sk=128, D=64, scale=0.125,
+                causal=0, dtype=fa.FA_FP16)
+    args.update(kw)
+    return fa.fa_fwd(*args.values())
+
+
+def bwd(**kw):
+    args = dict(q=A, k=A, v=A, o=A, lse=A, dO=A, dq=A, dk=A, dv=A, B=1, H=2, Sq=128, Sk=128, D=64,
+                scale=0.125, causal=0, dtype=fa.FA_FP16, ws=A, ws_bytes=1 << 30)
+    args.update(kw)
+    return fa.fa_bwd(*args.values())
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), -1), (dict(o=None), -1), (dict(lse=None), -1),
+    (dict(B=0), -1), (dict(H=-1), -1), (dict(Sq=0), -1), (dict(Sk=0), -1),
+    (dict(scale=0.0), -1), (dict(scale=-1.0), -1), (dict(scale=float("nan")), -1), (dict(scale=float("inf")), -1),
+    (dict(causal=2), -1),
+    (dict(D=32), -2), (dict(D=96), -2), (dict(D=256), -2), (dict(dtype=2), -2), (dict(dtype=-1), -2),
+    (dict(q=A + 8), -3), (dict(v=A + 2), -3), (dict(o=A + 4), -3), (dict(lse=A + 2), -3),
+    (dict(B=1 << 16, H=1 << 16, Sq=1 << 10), -1),
+])
+def test_fwd_rejects(fa_lib, kw, code):
+    assert fwd(**kw) == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dO=None), -1), (dict(dq=None), -1), (dict(dk=None), -1), (dict(dv=None), -1), (dict(lse=None), -1),
+    (dict(D=80), -2), (dict(dtype=3), -2), (dict(dk=A + 8), -3), (dict(dO=A + 4), -3),
+    (dict(ws=None), -7), (dict(ws_bytes=100), -7), (dict(ws=A + 16), -3),
+])
+def test_bwd_rejects(fa_lib, kw, code):
+    assert bwd(**kw) == code
+
+
+def test_strided_views_checked(fa_lib):
+    t = fa.FaTensor(A, 3 * 512 * 12 * 64, 3 * 12 * 64, 64)
+    p = fa.FwdParams(t, t, t, t, A, 2, 12, 512, 512, 64, 0.125, 0, fa.FA_FP16)
+    bad = fa.FaTensor(A, 3 * 512 * 12 * 64, 3 * 12 * 64 + 4, 64)  # seq stride not a multiple of 8
+    p.k = bad
+    assert fa.fa_fwd_ex(p) == -3
+    p.k = fa.FaTensor(A, -1, 64, 64)
+    assert fa.fa_fwd_ex(p) == -1
+    assert fa_lib.fa_fwd_ex(None, None) == -1
+    assert fa_lib.fa_bwd_ex(None, None) == -1
+
+
+def test_torch_helpers_refuse_cpu_tensors(fa_lib):
+    import torch
+    q = torch.zeros(1, 8, 1, 64, dtype=torch.float16)
+    with pytest.raises(ValueError):
+        fa.forward(q, q, q)
+    with pytest.raises(TypeError):
+        fa.forward(q.float(), q.float(), q.float())
