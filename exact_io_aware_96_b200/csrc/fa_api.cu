@@ -126,6 +126,55 @@ int launch_fwd(const fa_fwd_params* p, cudaStream_t stream) {
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+template <int D, bool BF16>
+int launch_bwd(const fa_bwd_params* p, cudaStream_t stream) {
+  using L = fa::BwdLayout<D>;
+  static bool done[kMaxDevices] = {};
+  auto* kern = &fa::fa_bwd_main<D, BF16>;
+  int st = prepare(kern, L::SMEM_ALLOC, done);
+  if (st != FA_OK) return st;
+  CUtensorMap mq, mk, mv, mdo;
+  if ((st = make_map(&mq, p->q, p->B, p->Sq, p->H, D, p->dtype, L::BM)) != FA_OK) return st;
+  if ((st = make_map(&mk, p->k, p->B, p->Sk, p->H, D, p->dtype, L::BN)) != FA_OK) return st;
+  if ((st = make_map(&mv, p->v, p->B, p->Sk, p->H, D, p->dtype, L::BN)) != FA_OK) return st;
+  if ((st = make_map(&mdo, p->dO, p->B, p->Sq, p->H, D, p->dtype, L::BM)) != FA_OK) return st;
+  fa::BwdArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.o = p->o.ptr;
+  a.dO = p->dO.ptr;
+  a.lse = p->lse;
+  a.dq = p->dq.ptr;
+  a.dk = p->dk.ptr;
+  a.dv = p->dv.ptr;
+  a.Sq_pad = (p->Sq + 127) / 128 * 128;
+  const int64_t rows = int64_t(p->B) * p->H * a.Sq_pad;
+  a.dq_acc = static_cast<float*>(p->workspace);
+  a.dvec = a.dq_acc + rows * D;
+  a.lse2 = a.dvec + rows;
+  a.o_sb = p->o.stride_b, a.o_ss = p->o.stride_s, a.o_sh = p->o.stride_h;
+  a.do_sb = p->dO.stride_b, a.do_ss = p->dO.stride_s, a.do_sh = p->dO.stride_h;
+  a.dq_sb = p->dq.stride_b, a.dq_ss = p->dq.stride_s, a.dq_sh = p->dq.stride_h;
+  a.dk_sb = p->dk.stride_b, a.dk_ss = p->dk.stride_s, a.dk_sh = p->dk.stride_h;
+  a.dv_sb = p->dv.stride_b, a.dv_ss = p->dv.stride_s, a.dv_sh = p->dv.stride_h;
+  a.B = p->B;
+  a.H = p->H;
+  a.Sq = p->Sq;
+  a.Sk = p->Sk;
+  a.scale = p->scale;
+  a.scale_log2 = p->scale * 1.4426950408889634f;
+  a.causal = p->causal;
+  constexpr int G = D / 8;
+  const int64_t pre_threads = rows * G;
+  fa::fa_bwd_pre<D, BF16><<<unsigned((pre_threads + 255) / 256), 256, 0, stream>>>(a);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  const unsigned grid = unsigned(int64_t((p->Sk + L::BN - 1) / L::BN) * p->B * p->H);
+  kern<<<grid, L::kThreads, L::SMEM_ALLOC, stream>>>(mq, mk, mv, mdo, a);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  const int64_t dq_threads = int64_t(p->B) * p->H * p->Sq * G;
+  fa::fa_bwd_dq<D, BF16><<<unsigned((dq_threads + 255) / 256), 256, 0, stream>>>(a);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" {
@@ -183,7 +232,7 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
 size_t fa_bwd_workspace_size(int B, int H, int Sq, int D) {
   if (B < 1 || H < 1 || Sq < 1 || D < 1) return 0;
   const uint64_t rows = uint64_t(B) * H * ((uint64_t(Sq) + 127) / 128 * 128);
-  const uint64_t bytes = rows * uint64_t(D) * 4 + rows * 4;
+  const uint64_t bytes = rows * (uint64_t(D) + 2) * 4;  // dq accumulator, Dvec, LSE * log2(e)
   if (bytes > (uint64_t(1) << 50)) return 0;
   return size_t(bytes);
 }
@@ -201,7 +250,8 @@ int fa_bwd_ex(const fa_bwd_params* p, fa_stream_t stream) {
   if (p->workspace == nullptr || p->workspace_bytes < need || need == 0) return FA_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(p->workspace) & 255u) return FA_ERR_MISALIGNED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  return fa::launch_bwd(p, s);
+  if (p->D == 64) return p->dtype == FA_BF16 ? launch_bwd<64, true>(p, s) : launch_bwd<64, false>(p, s);
+  return p->dtype == FA_BF16 ? launch_bwd<128, true>(p, s) : launch_bwd<128, false>(p, s);
 }
 
 int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO, void* dq,

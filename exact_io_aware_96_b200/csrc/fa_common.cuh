@@ -51,6 +51,15 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatil
   }
 }
 
+// Bounded wait used only on wind-down paths, to let copies or MMAs already in
+// flight land before the CTA exits or releases tensor memory.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = sm100::globaltimer_ns();
+  while (!sm100::mbar_try_wait(bar, parity)) {
+    if (sm100::globaltimer_ns() - t0 > 500000000ull) break;
+  }
+}
+
 struct FwdArgs {
   void* o;
   float* lse;
@@ -69,7 +78,8 @@ struct BwdArgs {
   void* dk;
   void* dv;
   float* dq_acc;  // fp32 [B, H, Sq_pad, D]
-  float* dvec;    // fp32 [B, H, Sq_pad]
+  float* dvec;    // fp32 [B, H, Sq_pad]: sum_d dO_id O_id
+  float* lse2;    // fp32 [B, H, Sq_pad]: LSE * log2(e); +inf where no key or padding
   int64_t o_sb, o_ss, o_sh;
   int64_t do_sb, do_ss, do_sh;
   int64_t dq_sb, dq_ss, dq_sh;

@@ -66,14 +66,6 @@ __device__ __forceinline__ int fwd_kv_blocks(int r0, int Sq, int Sk, int causal)
   return min(nk, last / 128 + 1);
 }
 
-// Bounded wait used only on the abort path to let in-flight copies land.
-__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
-  const uint64_t t0 = sm100::globaltimer_ns();
-  while (!sm100::mbar_try_wait(bar, parity)) {
-    if (sm100::globaltimer_ns() - t0 > 500000000ull) break;
-  }
-}
-
 template <int D, bool BF16>
 __global__ void __launch_bounds__(320, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,

@@ -136,9 +136,11 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o,
 /* Backward on strided views. Same semantics. */
 int fa_bwd_ex(const fa_bwd_params* p, fa_stream_t stream);
 
-/* Bytes of device workspace fa_bwd needs: an fp32 dq accumulator and the fp32
-   row terms Dvec_i = sum_d dO_id O_id, each padded to whole 128-row blocks.
-   Returns 0 for sizes < 1 or on overflow. */
+/* Bytes of device workspace fa_bwd needs: an fp32 dq accumulator
+   [B, H, Sq_pad, D], the fp32 row terms Dvec_i = sum_d dO_id O_id
+   [B, H, Sq_pad] and the fp32 logsumexp in base 2 [B, H, Sq_pad], where
+   Sq_pad is Sq rounded up to a multiple of 128. Returns 0 for sizes < 1 or on
+   overflow. */
 size_t fa_bwd_workspace_size(int B, int H, int Sq, int D);
 
 /* Synchronises the current device, returns the status word recorded by

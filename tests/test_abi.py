@@ -34,9 +34,9 @@ def test_version_and_strerror(fa_lib):
 
 
 def test_workspace_size(fa_lib):
-    # dq accumulator (fp32, rows padded to 128) + Dvec (fp32)
-    assert fa.fa_bwd_workspace_size(1, 2, 128, 64) == 2 * 128 * 64 * 4 + 2 * 128 * 4
-    assert fa.fa_bwd_workspace_size(2, 12, 2000, 64) == 24 * 2048 * 64 * 4 + 24 * 2048 * 4
+    # dq accumulator (fp32, rows padded to 128) + Dvec + base-2 LSE (fp32)
+    assert fa.fa_bwd_workspace_size(1, 2, 128, 64) == 2 * 128 * 64 * 4 + 2 * 2 * 128 * 4
+    assert fa.fa_bwd_workspace_size(2, 12, 2000, 64) == 24 * 2048 * 64 * 4 + 2 * 24 * 2048 * 4
     assert fa.fa_bwd_workspace_size(0, 1, 1, 64) == 0
     assert fa.fa_bwd_workspace_size(1, 1, -5, 64) == 0
 
