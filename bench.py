@@ -1,0 +1,393 @@
+#!/usr/bin/env python
+"""Throughput of exact attention forward + backward on B200 through libfa.so.
+
+One step = one pass of the whole path on one batch of synthetic input:
+fa_fwd (fused forward) then fa_bwd (preprocess, dK/dV/dQ main kernel, dQ
+convert) on the headline workload c4: B=1, H=8, S=8192, D=128, bf16, causal.
+Throughput counts the algorithmic dense-contraction FLOPs, 4*B*H*S*S*D halved
+for causal in the forward and 2.5x that in the backward (the backward's five
+matrix products against the forward's two).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs under torchrun, one process per GPU: every rank processes its own
+batch (weak scaling; attention heads are independent, so there is no
+collective on the data path). Rank 0 prints one JSON line.
+
+``--impl reference`` times the fp64 CPU oracle on the same workload (one head
+of it per step) on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd/bwd TFLOP/s (bf16, causal, S=8K, d=128) and % of B200 dense peak"
+NOMINAL_BF16_TFLOPS = 2250.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ----------------------------------------------------------------- helpers
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def rank_batch_slice(global_batch: int, world: int, rank: int):
+    """Batch rows [lo, hi) owned by `rank`: contiguous, sizes differ by at most one."""
+    base, extra = divmod(global_batch, world)
+    lo = rank * base + min(rank, extra)
+    return lo, lo + base + (1 if rank < extra else 0)
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    """Max of a per-rank scalar over the process group (identity without one)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "exact_io_aware_96_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML every `period` s."""
+
+    def __init__(self, index: int, period: float = 0.01):
+        self.index, self.period = index, period
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+
+    def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            names = {
+                "hw_slowdown": getattr(pynvml, "nvmlClocksEventReasonHwSlowdown", 0x8),
+                "hw_thermal_slowdown": getattr(pynvml, "nvmlClocksEventReasonHwThermalSlowdown", 0x40),
+                "sw_thermal_slowdown": getattr(pynvml, "nvmlClocksEventReasonSwThermalSlowdown", 0x20),
+                "sw_power_cap": getattr(pynvml, "nvmlClocksEventReasonSwPowerCap", 0x4),
+                "hw_power_brake_slowdown": getattr(pynvml, "nvmlClocksEventReasonHwPowerBrakeSlowdown", 0x80),
+            }
+
+            def run():
+                while not self._stop.is_set():
+                    try:
+                        self.samples.append(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM))
+                        try:
+                            r = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                        except AttributeError:
+                            r = pynvml.nvmlDeviceGetCurrentClocksThrottleReasons(h)
+                        for n, bit in names.items():
+                            if r & bit:
+                                self.reasons.add(n)
+                    except Exception:
+                        pass
+                    time.sleep(self.period)
+
+            self._t = threading.Thread(target=run, daemon=True)
+            self._t.start()
+        except Exception as e:  # NVML missing: report no samples
+            self.error = repr(e)
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._t is not None:
+            self._t.join()
+
+    def summary(self):
+        busy = [s for s in self.samples if self.max_mhz and s > 0.3 * self.max_mhz] or self.samples
+        return {"sm_mhz": statistics.median(busy) if busy else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def flops(w, causal):
+    return w.fwd_flops(causal), w.bwd_flops(causal)
+
+
+# ------------------------------------------------------------ CPU baseline
+def oracle_sample(w, causal, inp64, heads, budget_s=None):
+    """Run the fp64 oracle (forward + backward) head by head; stop after
+    `heads` heads or once `budget_s` seconds have passed. Returns (flops, s, n)."""
+    import oracle
+    q, k, v, do = inp64
+    done, t0 = 0, time.perf_counter()
+    for h in range(heads):
+        oracle.attention_head(q, k, v, do, w.scale, causal, 0, h)
+        done += 1
+        if budget_s is not None and time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    ff, fb = flops(w, causal)
+    return (ff + fb) / (w.B * w.H) * done, dt, done
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [p.get("num_threads") for p in threadpool_info() if p.get("user_api") == "blas"]
+        return int(max(n)) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def host_inputs64(w):
+    import torch
+    from exact_io_aware_96_b200.inputs import make_inputs
+    inp = make_inputs(w)
+    return [inp[n].to(torch.float64).numpy() for n in ("q", "k", "v", "do")]
+
+
+# --------------------------------------------------------------- our arm
+def run_ours(args, w, causal):
+    import torch
+    import torch.distributed as dist
+    from exact_io_aware_96_b200 import fa
+    from exact_io_aware_96_b200.inputs import make_inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    fa.lib()  # fail loudly if the library is missing
+
+    # Each rank owns rows [lo, hi) of a global batch of world * B; the draw
+    # for rank r uses seed + r so that ranks hold different data.
+    lo, hi = rank_batch_slice(w.B * world, world, rank)
+    inp = make_inputs(w, B=hi - lo) if rank == 0 else make_inputs(
+        type(w)(**{**w.__dict__, "seed": w.seed + rank}), B=hi - lo)
+    q, k, v, do = (inp[n].to(dev) for n in ("q", "k", "v", "do"))
+    B, S, H, D = q.shape
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, S), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = fa.workspace_for(B, H, S, D, dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        fa.forward(q, k, v, causal=causal, scale=w.scale, out=o, lse=lse, stream=stream)
+        fa.backward(q, k, v, o, lse, do, causal=causal, scale=w.scale, dq=dq, dk=dk, dv=dv,
+                    workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    st, detail = fa.fa_last_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} {detail} after warm-up")
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    with ClockSampler(local) as clocks:
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        wall0 = time.perf_counter()
+        for i in range(args.steps):
+            flush.zero_()  # evict the inputs from L2 (outside the timed events)
+            ev[i][0].record(stream)
+            fa.forward(q, k, v, causal=causal, scale=w.scale, out=o, lse=lse, stream=stream)
+            ev[i][1].record(stream)
+            fa.backward(q, k, v, o, lse, do, causal=causal, scale=w.scale, dq=dq, dk=dk, dv=dv,
+                        workspace=ws, stream=stream)
+            ev[i][2].record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        wall = time.perf_counter() - wall0
+    st, detail = fa.fa_last_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} {detail} in the timed region")
+
+    t_fwd = sum(e[0].elapsed_time(e[1]) for e in ev) / 1e3
+    t_bwd = sum(e[1].elapsed_time(e[2]) for e in ev) / 1e3
+    t_dev = max_over_ranks(t_fwd + t_bwd, dev)
+    t_fwd_max = max_over_ranks(t_fwd, dev)
+    t_bwd_max = max_over_ranks(t_bwd, dev)
+
+    ff, fb = flops(w, causal)
+    ff *= (hi - lo) / w.B
+    fb *= (hi - lo) / w.B
+    total_flops = (ff + fb) * args.steps * world
+    value = total_flops / t_dev / 1e12
+    fwd_tf = ff * args.steps / t_fwd_max / 1e12
+    bwd_tf = fb * args.steps / t_bwd_max / 1e12
+
+    # ---- end to end through the public API: pinned host inputs -> device ->
+    # fa.forward + fa.backward -> outputs back to pinned host memory.
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv, hdo = (t.cpu().pin_memory() for t in (q, k, v, do))
+        ho, hl = torch.empty_like(o, device="cpu").pin_memory(), torch.empty_like(lse, device="cpu").pin_memory()
+        hdq, hdk, hdv = (torch.empty_like(t, device="cpu").pin_memory() for t in (dq, dk, dv))
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo))
+        d2h = sum(t.numel() * t.element_size() for t in (ho, hl, hdq, hdk, hdv))
+
+        def e2e_step():
+            for src, dst in ((hq, q), (hk, k), (hv, v), (hdo, do)):
+                dst.copy_(src, non_blocking=True)
+            step()
+            for src, dst in ((o, ho), (lse, hl), (dq, hdq), (dk, hdk), (dv, hdv)):
+                dst.copy_(src, non_blocking=True)
+
+        for _ in range(max(1, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize()
+        n_e2e = max(3, min(args.steps, 50))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        e0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        t_e2e = max_over_ranks(e0.elapsed_time(e1) / 1e3, dev)
+        e2e = {"value": (ff + fb) * n_e2e * world / t_e2e / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e}
+
+    peaks, peaks_src = load_peaks()
+    timed_s = t_fwd + t_bwd
+    sustained = timed_s > 1.0
+    peak_tf = peaks.get("bf16_tflops_sustained" if sustained else "bf16_tflops")
+    # Dominant call of a step: the one with the larger share of device time.
+    if t_bwd >= t_fwd:
+        dom, dom_flops, dom_t = "fa_bwd (fa_bwd_pre + fa_bwd_main + fa_bwd_dq)", fb, t_bwd_max / args.steps
+    else:
+        dom, dom_flops, dom_t = "fa_fwd_kernel", ff, t_fwd_max / args.steps
+    achieved = dom_flops / dom_t / 1e12
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tpath):
+        with open(tpath) as f:
+            tr = json.load(f)
+        ent = tr.get(dom.split(" ")[0])
+        if ent and ent.get("source_hash") == kernel_source_hash():
+            traffic = ent.get("bytes_per_launch")
+
+    result = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": t_dev / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{w.name}: B={w.B} H={w.H} S={w.S} D={w.D} bf16 causal={causal}, "
+                               "forward + backward per step",
+                   "global_batch": w.B * world, "seq_len": w.S, "heads": w.H, "head_dim": w.D,
+                   "causal": causal, "parallelism": f"dp{world} (independent heads, no collective)",
+                   "l2": "flushed before every step (256 MiB write, outside the timed events)"},
+        "fwd_tflops": fwd_tf, "bwd_tflops": bwd_tf,
+        "fwd_us": t_fwd_max / args.steps * 1e6, "bwd_us": t_bwd_max / args.steps * 1e6,
+        "pct_of_nominal_2250": {"fwd": 100 * fwd_tf / NOMINAL_BF16_TFLOPS, "bwd": 100 * bwd_tf / NOMINAL_BF16_TFLOPS},
+        "pct_of_measured_bf16": {"fwd": 100 * fwd_tf / peaks["bf16_tflops"], "bwd": 100 * bwd_tf / peaks["bf16_tflops"],
+                                 "peak": peaks["bf16_tflops"]},
+        "roofline": {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
+                     "frac": achieved / peak_tf, "traffic": traffic,
+                     "peak_source": f"{peaks_src} {'bf16_tflops_sustained' if sustained else 'bf16_tflops'}"},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clocks.summary(),
+        "wall_s_timed_region": wall,
+        "e2e": e2e,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        inp64 = host_inputs64(w)
+        fl, dt, n = oracle_sample(w, causal, inp64, w.H, budget_s=args.cpu_budget)
+        result["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
+                                  "kind": "oracle",
+                                  "sample": f"{n} of {w.H} heads of {w.name} (b=0), fp64 forward + backward, "
+                                            f"{dt:.1f} s"}
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return result if rank == 0 else None
+
+
+# --------------------------------------------------------- reference arm
+def run_reference(args, w, causal):
+    """The oracle as it stands, on the host cores: one head of the workload
+    (forward + backward, fp64) per step. Rank 0 only."""
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return None
+    inp64 = host_inputs64(w)
+    for i in range(args.warmup):
+        oracle_sample(w, causal, [a for a in inp64], 1)
+    t0 = time.perf_counter()
+    total = 0.0
+    for i in range(args.steps):
+        fl, _, _ = oracle_sample(w, causal, inp64, 1)
+        total += fl
+    dt = time.perf_counter() - t0
+    value = total / dt / 1e12
+    cores = blas_threads()
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{w.name}: B={w.B} H={w.H} S={w.S} D={w.D} causal={causal}; one head per step",
+                   "global_batch": w.B, "seq_len": w.S, "heads": 1, "head_dim": w.D, "causal": causal},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": f"one head of {w.name} per step (fp64 forward + backward, numpy/OpenBLAS)"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="c4")
+    ap.add_argument("--causal", type=int, choices=[0, 1], default=None,
+                    help="override the workload's (first) mask setting")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "ours":
+        ap.error("--warmup must be >= 3")
+    from exact_io_aware_96_b200.inputs import WORKLOADS
+    w = WORKLOADS[args.workload]
+    causal = bool(w.causal[0] if args.causal is None else args.causal)
+    res = run_reference(args, w, causal) if args.impl == "reference" else run_ours(args, w, causal)
+    if res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,102 @@
+"""Backward parity on the GPU: libfa.so (through the C ABI) vs the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from exact_io_aware_96_b200 import fa
+from exact_io_aware_96_b200.inputs import WORKLOADS, make_inputs, random_case, sample_rows
+from tests.parity import check_grad, check_o_lse, full_check, np64, rel_l2, run_bwd, run_fwd
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("S", [1, 7, 63, 64, 65, 127, 128, 129, 200, 256, 257, 640])
+def test_bwd_square(D, dtype, causal, S):
+    full_check(random_case(1, 2, S, S, D, dtype, 2000 + S), causal, what=f"S{S} D{D} {dtype} c{causal}")
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("Sq,Sk", [(1, 300), (100, 37), (129, 700), (700, 129), (300, 1), (256, 512), (513, 255)])
+def test_bwd_rectangular(D, causal, Sq, Sk):
+    full_check(random_case(2, 3, Sq, Sk, D, torch.bfloat16, 31 + Sq + Sk), causal,
+               what=f"Sq{Sq} Sk{Sk} D{D} c{causal}")
+
+
+@pytest.mark.parametrize("scale", [0.02, 0.5])
+def test_bwd_scale(scale):
+    full_check(random_case(1, 2, 300, 300, 128, torch.float16, 9), True, scale=scale, what=f"scale {scale}")
+
+
+def test_bwd_wide_scores():
+    full_check(random_case(1, 2, 700, 700, 128, torch.bfloat16, 13, qk_std=2.0), True, what="wide")
+
+
+@pytest.mark.parametrize("name", ["c1", "c3", "c3r"])
+def test_bwd_workloads_full(name):
+    w = WORKLOADS[name]
+    inp = make_inputs(w)
+    for causal in w.causal:
+        full_check(inp, causal, scale=w.scale, what=f"{name} causal={causal}")
+
+
+def test_bwd_packed_qkv():
+    """c2: q, k, v are strided views into one [B, S, 3, H, D] tensor; the
+    gradients are written into the matching views of one dqkv tensor."""
+    w = WORKLOADS["c2"]
+    inp = make_inputs(w)
+    qkv = inp["qkv"].cuda()
+    do = inp["do"].cuda()
+    q, k, v = qkv[:, :, 0], qkv[:, :, 1], qkv[:, :, 2]
+    o, lse = run_fwd(q, k, v, False, w.scale)
+    dqkv = torch.full_like(qkv, float("nan"))
+    fa.backward(q, k, v, o, lse, do, causal=False, scale=w.scale,
+                dq=dqkv[:, :, 0], dk=dqkv[:, :, 1], dv=dqkv[:, :, 2])
+    torch.cuda.synchronize()
+    qn, kn, vn, don = np64(inp["q"]), np64(inp["k"]), np64(inp["v"]), np64(inp["do"])
+    o_ref, lse_ref = oracle.attention_forward(qn, kn, vn, w.scale, False)
+    check_o_lse(np64(o), np64(lse), o_ref, lse_ref, w.dtype, "c2 fwd")
+    dq_r, dk_r, dv_r, _ = oracle.attention_backward(qn, kn, vn, don, w.scale, False)
+    g = np64(dqkv)
+    for j, (name, ref) in enumerate((("dq", dq_r), ("dk", dk_r), ("dv", dv_r))):
+        check_grad(g[:, :, j], ref, f"c2 {name}")
+
+
+def test_bwd_repeatable_dk_dv():
+    """dK and dV have a fixed summation order; dQ is accumulated with atomics."""
+    c = random_case(1, 2, 900, 900, 128, torch.bfloat16, 17)
+    q, k, v, do = (c[n].cuda() for n in ("q", "k", "v", "do"))
+    o, lse = run_fwd(q, k, v, True)
+    a = run_bwd(q, k, v, o, lse, do, True)
+    b = run_bwd(q, k, v, o, lse, do, True)
+    assert torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])
+    assert rel_l2(np64(a[0]), np64(b[0])) < 1e-3
+
+
+@pytest.mark.parametrize("name", ["c4", "c5"])
+def test_bwd_workloads_sampled(name):
+    """Full-size launch. dQ checked on sampled rows of every head; dK and dV
+    need every query row, so they are checked in full on the first and last head."""
+    w = WORKLOADS[name]
+    inp = make_inputs(w)
+    dev = {n: inp[n].cuda() for n in ("q", "k", "v", "do")}
+    rows = sample_rows(w.S, 128, 118, w.seed)
+    qn, kn, vn, don = (np64(inp[n]) for n in ("q", "k", "v", "do"))
+    for causal in w.causal:
+        o, lse = run_fwd(dev["q"], dev["k"], dev["v"], causal, w.scale)
+        dq, dk, dv = run_bwd(dev["q"], dev["k"], dev["v"], o, lse, dev["do"], causal, w.scale)
+        dq, dk, dv = np64(dq), np64(dk), np64(dv)
+        got, ref = [], []
+        for h in range(w.H):
+            got.append(dq[0, rows, h])
+            ref.append(oracle.attention_backward_dq_rows(qn, kn, vn, don, w.scale, causal, 0, h, rows))
+        check_grad(np.stack(got), np.stack(ref), f"{name} dq rows causal={causal}")
+        for h in (0, w.H - 1):
+            hd = oracle.attention_head(qn, kn, vn, don, w.scale, causal, 0, h)
+            check_grad(dk[0, :, h], hd["dk"], f"{name} dk h{h} causal={causal}")
+            check_grad(dv[0, :, h], hd["dv"], f"{name} dv h{h} causal={causal}")
+            del hd
