@@ -66,10 +66,17 @@ def max_over_ranks(x: float, device=None) -> float:
     return float(t.item())
 
 
-def kernel_source_hash() -> str:
+KERNEL_SOURCES = {
+    "fa_bwd": ["fa_bwd.cuh", "fa_common.cuh", "sm100.cuh"],
+    "fa_fwd_kernel": ["fa_fwd.cuh", "fa_common.cuh", "sm100.cuh"],
+}
+
+
+def kernel_source_hash(kernel: str) -> str:
+    """Hash of the sources a kernel is built from (to tell stale counters)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "exact_io_aware_96_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in KERNEL_SOURCES[kernel]:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
@@ -78,7 +85,7 @@ def kernel_source_hash() -> str:
 class ClockSampler:
     """Samples SM clock and throttle reasons through NVML every `period` s."""
 
-    def __init__(self, index: int, period: float = 0.01):
+    def __init__(self, index: int, period: float = 0.002):
         self.index, self.period = index, period
         self.samples, self.reasons = [], set()
         self.max_mhz = None
@@ -295,8 +302,9 @@ def run_ours(args, w, causal):
     if os.path.exists(tpath):
         with open(tpath) as f:
             tr = json.load(f)
-        ent = tr.get(dom.split(" ")[0])
-        if ent and ent.get("source_hash") == kernel_source_hash():
+        key = dom.split(" ")[0]
+        ent = tr.get(key)
+        if ent and ent.get("source_hash") == kernel_source_hash(key):
             traffic = ent.get("bytes_per_launch")
 
     result = {
@@ -369,7 +377,7 @@ def run_reference(args, w, causal):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="c4")
