@@ -177,6 +177,35 @@ int launch_bwd(const fa_bwd_params* p, cudaStream_t stream) {
 
 }  // namespace
 
+// Device scratch of fa_bwd_noalloc: a file-scope array, so the library never
+// allocates for it. Host code cannot use the name as an address; its device
+// address is looked up once per device (noalloc_scratch) and passed to the
+// kernels like a caller's workspace.
+constexpr size_t kNoAllocScratchBytes = FA_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device; set up on the
+// first call per device (cudaGetSymbolAddress), cached afterwards.
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) return FA_ERR_CUDA;
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return FA_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 int fa_version(void) { return 100; }
@@ -191,6 +220,7 @@ const char* fa_strerror(int s) {
     case FA_ERR_TIMEOUT: return "device-side pipeline wait exceeded its time limit";
     case FA_ERR_NOT_IMPLEMENTED: return "not implemented";
     case FA_ERR_WORKSPACE: return "workspace missing or smaller than fa_bwd_workspace_size()";
+    case FA_ERR_SCRATCH_LIMIT: return "fa_bwd_noalloc: the problem needs more scratch than FA_NOALLOC_SCRATCH_BYTES (64 MiB)";
     default: return "unknown status";
   }
 }
@@ -278,6 +308,45 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
   p.dtype = dtype;
   p.workspace = workspace;
   p.workspace_bytes = workspace_bytes;
+  return fa_bwd_ex(&p, stream);
+}
+
+int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                   void* dq, void* dk, void* dv, int B, int H, int Sq, int Sk, int D, float scale, int causal,
+                   int dtype, fa_stream_t stream) {
+  fa_bwd_params p;
+  std::memset(&p, 0, sizeof(p));
+  p.q = dense(q, Sq, H, D);
+  p.k = dense(k, Sk, H, D);
+  p.v = dense(v, Sk, H, D);
+  p.o = dense(o, Sq, H, D);
+  p.dO = dense(dO, Sq, H, D);
+  p.lse = lse;
+  p.dq = dense(dq, Sq, H, D);
+  p.dk = dense(dk, Sk, H, D);
+  p.dv = dense(dv, Sk, H, D);
+  p.B = B;
+  p.H = H;
+  p.Sq = Sq;
+  p.Sk = Sk;
+  p.D = D;
+  p.scale = scale;
+  p.causal = causal;
+  p.dtype = dtype;
+  // Every argument check comes before the first CUDA call.
+  int st = check_common(B, H, Sq, Sk, D, scale, causal, dtype);
+  if (st != FA_OK) return st;
+  const fa_tensor* views[8] = {&p.q, &p.k, &p.v, &p.o, &p.dO, &p.dq, &p.dk, &p.dv};
+  for (const fa_tensor* t : views)
+    if ((st = check_view(*t)) != FA_OK) return st;
+  if (lse == nullptr) return FA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(lse) & 3u) return FA_ERR_MISALIGNED;
+  const size_t need = fa_bwd_workspace_size(B, H, Sq, D);
+  if (need == 0 || need > kNoAllocScratchBytes) return FA_ERR_SCRATCH_LIMIT;
+  void* scratch = nullptr;
+  if ((st = noalloc_scratch(&scratch)) != FA_OK) return st;
+  p.workspace = scratch;
+  p.workspace_bytes = kNoAllocScratchBytes;
   return fa_bwd_ex(&p, stream);
 }
 

@@ -20,8 +20,10 @@ FA_OK = 0
 STATUS = {
     0: "FA_OK", -1: "FA_ERR_INVALID_ARG", -2: "FA_ERR_UNSUPPORTED", -3: "FA_ERR_MISALIGNED",
     -4: "FA_ERR_CUDA", -5: "FA_ERR_TIMEOUT", -6: "FA_ERR_NOT_IMPLEMENTED", -7: "FA_ERR_WORKSPACE",
+    -8: "FA_ERR_SCRATCH_LIMIT",
 }
-EXPORTED = ("fa_fwd", "fa_fwd_ex", "fa_bwd", "fa_bwd_ex", "fa_bwd_workspace_size",
+FA_NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
+EXPORTED = ("fa_fwd", "fa_fwd_ex", "fa_bwd", "fa_bwd_ex", "fa_bwd_noalloc", "fa_bwd_workspace_size",
             "fa_last_device_status", "fa_strerror", "fa_version")
 
 
@@ -73,6 +75,8 @@ def lib():
         L.fa_bwd.restype = i
         L.fa_bwd_ex.argtypes = [ctypes.POINTER(BwdParams), vp]
         L.fa_bwd_ex.restype = i
+        L.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp]
+        L.fa_bwd_noalloc.restype = i
         L.fa_bwd_workspace_size.argtypes = [i, i, i, i]
         L.fa_bwd_workspace_size.restype = sz
         L.fa_last_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
@@ -102,6 +106,12 @@ def fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, Sq, Sk, D, scale, causal, dtyp
 
 def fa_bwd_ex(params: BwdParams, stream=0) -> int:
     return lib().fa_bwd_ex(ctypes.byref(params), stream)
+
+
+def fa_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, B, H, Sq, Sk, D, scale, causal, dtype, stream=0) -> int:
+    """Backward with the library's built-in scratch instead of a workspace
+    (for callers that cannot allocate device memory; see include/fa.h)."""
+    return lib().fa_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, B, H, Sq, Sk, D, scale, causal, dtype, stream)
 
 
 def fa_bwd_workspace_size(B, H, Sq, D) -> int:

@@ -77,8 +77,13 @@ typedef enum {
   FA_ERR_CUDA = -4,            /* a CUDA runtime/driver call failed */
   FA_ERR_TIMEOUT = -5,         /* a device-side pipeline wait ran out (fa_last_device_status) */
   FA_ERR_NOT_IMPLEMENTED = -6, /* reserved */
-  FA_ERR_WORKSPACE = -7        /* workspace pointer null or smaller than fa_bwd_workspace_size */
+  FA_ERR_WORKSPACE = -7,       /* workspace pointer null or smaller than fa_bwd_workspace_size */
+  FA_ERR_SCRATCH_LIMIT = -8    /* fa_bwd_noalloc: problem needs more than FA_NOALLOC_SCRATCH_BYTES */
 } fa_status;
+
+/* Size of the built-in device scratch buffer of fa_bwd_noalloc (64 MiB per
+   device that loads the library). */
+#define FA_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
 
 /* A strided [B, S, H, D] view: element strides for batch, sequence and head;
    the head_dim axis has stride 1. */
@@ -135,6 +140,36 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o,
 
 /* Backward on strided views. Same semantics. */
 int fa_bwd_ex(const fa_bwd_params* p, fa_stream_t stream);
+
+/* Backward that allocates nothing and takes no workspace. Not a method step:
+   the pages have no counterpart; it exists for callers that cannot allocate
+   device memory themselves, such as code running inside a host application
+   that reserves all device memory up front and hands out only input and
+   output buffers, plug-in interfaces with no way to ask for a workspace, or
+   latency-critical code that must not call cudaMalloc (which may synchronise
+   the device).
+   Same arguments, semantics and results as fa_bwd, except that the scratch
+   (the fp32 dq accumulator, Dvec and the base-2 logsumexp) lives in one
+   static device array of FA_NOALLOC_SCRATCH_BYTES inside the library,
+   reserved on every device that loads it until the process exits. Problems
+   whose fa_bwd_workspace_size() exceeds that size return
+   FA_ERR_SCRATCH_LIMIT (about B*H*Sq*(D+2)*4 bytes; B*H = 8, Sq = 8192,
+   D = 128 needs 34 MB). No cudaMalloc, cudaFree or other allocating call is
+   made.
+   Set-up: the first call on a device (the current device) looks up the
+   array's device address with cudaGetSymbolAddress and caches it; make that
+   first call before any stream capture on that device. Later calls only
+   launch kernels.
+   Sharing: every call on a device uses the same array. Each call rewrites all
+   of the scratch it reads (the accumulator is zeroed by the call's first
+   kernel), so leftovers of earlier calls do not matter, but two calls that
+   run at the same time on one device (different streams, or host threads
+   without ordering between them) race on the array and give wrong results:
+   order them on one stream or with events. */
+int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                   const float* lse, const void* dO, void* dq, void* dk,
+                   void* dv, int B, int H, int Sq, int Sk, int D, float scale,
+                   int causal, int dtype, fa_stream_t stream);
 
 /* Bytes of device workspace fa_bwd needs: an fp32 dq accumulator
    [B, H, Sq_pad, D], the fp32 row terms Dvec_i = sum_d dO_id O_id
