@@ -137,6 +137,7 @@ int launch_bwd(const fa_bwd_params* p, cudaStream_t stream) {
   if ((st = make_map(&mq, p->q, p->B, p->Sq, p->H, D, p->dtype, L::BM)) != FA_OK) return st;
   if ((st = make_map(&mk, p->k, p->B, p->Sk, p->H, D, p->dtype, L::BN)) != FA_OK) return st;
   if ((st = make_map(&mv, p->v, p->B, p->Sk, p->H, D, p->dtype, L::BN)) != FA_OK) return st;
+  static_assert(L::BM == 128 && L::BN == 128, "tensor maps assume 128-row boxes");
   if ((st = make_map(&mdo, p->dO, p->B, p->Sq, p->H, D, p->dtype, L::BM)) != FA_OK) return st;
   fa::BwdArgs a;
   std::memset(&a, 0, sizeof(a));

@@ -22,15 +22,22 @@
 // dV = P^T dO, dP = dO V^T, dX = P (dP - rowsum(P dP)), dQ = scale dX K,
 // dK = scale dX^T Q, and rowsum(P dP)_i = sum_d dO_id O_id.
 //
-// Main kernel, warp roles (320 threads):
-//   warps 0-3  one key row per thread: P^T, dS^T; at the end dK
-//   warps 4-7  read the dQ block from TMEM, add it into the accumulator; at the end dV
-//   warp  8    TMA loader: K, V once; Q_i, dO_i, lse2_i, Dvec_i per query block
-//   warp  9    MMA issuer
-// D = 128 uses 64-row query blocks and two S^T/dP^T buffers so the softmax of
-// block i+1 overlaps the products of block i; dQ is computed transposed
-// (dQ^T = K^T dS^T, M = head_dim) into the dP^T buffer it follows. D = 64 uses
-// 128-row query blocks, one buffer, and dQ = dS K into its own columns.
+// Main kernel, warp roles (448 threads):
+//   warps 0-7   P^T and dS^T, one key row per thread; warps 0-3 take query
+//               columns [0, 64), warps 4-7 [64, 128). At the end warps 0-3
+//               write dK and warps 4-7 write dV.
+//   warps 8-11  read the dQ block out of TMEM and add it into the fp32
+//               accumulator (D = 128: dQ^T, one head_dim index per thread, so
+//               a warp's reductions hit one 128-byte line per query)
+//   warp  12    TMA loader: K, V once; Q_i, dO_i, lse2_i, Dvec_i per query block
+//   warp  13    MMA issuer
+// Blocks are 128 keys x 128 queries. Tensor memory: dK and dV accumulators,
+// X (S^T, then 16-bit P^T and dS^T written back by the softmax warps and used
+// as the TMEM A operand of dV += P^T dO and dK += dS^T Q) and Y (dP^T, then
+// dQ^T = K^T dS^T (D = 128) or dQ = dS K (D = 64), with dS^T staged in
+// 128-byte swizzled smem). The
+// MMA order per block i is dV(i), dK(i), S^T(i+1), dQ(i), dP^T(i+1), so the
+// softmax of block i+1 starts while dQ(i) and dP^T(i+1) run.
 //
 // Page legend: [P1] "Miniconda-Python3.9环境下使用FlashAttention优化训练";
 // [P2] "使用FlashAttention优化PyTorch模型注意力计算"; [P4] the FlashAttention-2
@@ -116,70 +123,85 @@ __global__ void __launch_bounds__(256) fa_bwd_dq(const BwdArgs a) {
 // ------------------------------------------------------------- main kernel
 template <int D>
 struct BwdLayout {
-  static constexpr int kThreads = 320;
-  static constexpr int BN = 128;                 // keys per CTA
-  static constexpr int BM = (D == 128) ? 64 : 128;  // query rows per block
-  static constexpr int NBUF = (D == 128) ? 2 : 1;   // S^T/dP^T buffers in TMEM
-  static constexpr int QS = 2;                   // Q/dO stages
-  static constexpr int KB = D / 64;              // 64-column blocks per row
-  static constexpr int KV_TILE = BN * D * 2;     // K or V tile bytes
-  static constexpr int KV_BLK = BN * 128;        // one [128 rows][64 cols] block
-  static constexpr int Q_TILE = BM * D * 2;      // Q or dO tile bytes
-  static constexpr int Q_BLK = BM * 128;         // one [BM rows][64 cols] block
-  static constexpr int DS_TILE = BN * BM * 2;    // dS^T tile bytes [128 keys][BM]
+  static constexpr int kThreads = 448;   // 14 warps
+  static constexpr int BN = 128;         // keys per CTA
+  static constexpr int BM = 128;         // query rows per block
+  static constexpr int QS = 2;           // Q/dO stages
+  // D = 128: dQ is computed transposed (TMEM lane = head_dim index), so each
+  // warp's reductions into the accumulator cover one contiguous 128-byte line.
+  static constexpr bool DQ_T = (D == 128);
+  static constexpr int KB = D / 64;      // 64-column blocks per row
+  static constexpr int TILE = 128 * D * 2;  // one K, V, Q or dO tile
+  static constexpr int BLK = 128 * 128;     // one [128 rows][64 cols] block
+  static constexpr int DS_TILE = 128 * 128 * 2;  // dS^T [128 keys][128 queries]
   static constexpr int OFF_K = 0;
-  static constexpr int OFF_V = OFF_K + KV_TILE;
-  static constexpr int OFF_Q = OFF_V + KV_TILE;
-  static constexpr int OFF_DO = OFF_Q + QS * Q_TILE;
-  static constexpr int OFF_DS = OFF_DO + QS * Q_TILE;
-  static constexpr int OFF_LSE = OFF_DS + 2 * DS_TILE;
+  static constexpr int OFF_V = OFF_K + TILE;
+  static constexpr int OFF_Q = OFF_V + TILE;
+  static constexpr int OFF_DO = OFF_Q + QS * TILE;
+  static constexpr int OFF_DS = OFF_DO + QS * TILE;
+  static constexpr int OFF_LSE = OFF_DS + DS_TILE;
   static constexpr int OFF_DVEC = OFF_LSE + QS * BM * 4;
   static constexpr int OFF_BAR = OFF_DVEC + QS * BM * 4;
-  // kv_full, q_full[QS], q_empty[QS], s_full[NBUF], ds_ready[NBUF], ds_free[2],
-  // dq_full[NBUF], dq_free[NBUF], mma_done, drain
-  static constexpr int NBAR = 1 + 2 * QS + 4 * NBUF + 2 + 2;
+  // kv_full, q_full[QS], q_empty[QS], sx_full, dp_full, p_ready, ds_ready,
+  // ds_free, dq_full, dq_free, mma_done, drain
+  static constexpr int NBAR = 1 + 2 * QS + 10;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int BYTES = OFF_MISC + 16;
-  static constexpr int SMEM_ALLOC = BYTES + 1024;
+  static constexpr int SMEM_MAX = 232448;
+  // 1024 bytes of slack to align the base when it fits; otherwise the kernel
+  // requires (and checks) a 1024-aligned dynamic shared memory base.
+  static constexpr int SMEM_ALLOC = (BYTES + 1024 <= SMEM_MAX) ? BYTES + 1024 : BYTES;
   static constexpr int TMEM_COLS = 512;
-  // TMEM columns
+  // TMEM columns: dK, dV accumulators; X holds S^T, then P^T and dS^T
+  // (16-bit); Y holds dP^T, then dQ.
   static constexpr int COL_DK = 0;
   static constexpr int COL_DV = D;
-  __host__ __device__ static constexpr int col_s(int b) { return 2 * D + b * 2 * BM; }
-  __host__ __device__ static constexpr int col_dp(int b) { return 2 * D + b * 2 * BM + BM; }
-  __host__ __device__ static constexpr int col_dq(int b) { return NBUF == 2 ? col_dp(b) : 2 * D + 2 * BM; }
+  static constexpr int COL_X = 2 * D;
+  static constexpr int COL_Y = 2 * D + 128;
+  // Softmax warpgroup g owns queries [64g, 64g + 64): it packs their P^T into
+  // X columns [64g, 64g + 32) and their dS^T into [64g + 32, 64g + 64).
+  __host__ __device__ static constexpr int col_p(int kk) { return COL_X + (kk >> 2) * 64 + (kk & 3) * 8; }
+  __host__ __device__ static constexpr int col_ds(int kk) { return COL_X + (kk >> 2) * 64 + 32 + (kk & 3) * 8; }
 };
 
 template <int D, bool BF16>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(448, 1)
     fa_bwd_main(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO, const BwdArgs a) {
   using L = BwdLayout<D>;
   using namespace sm100;
-  constexpr int BM = L::BM, NBUF = L::NBUF, QS = L::QS;
-  static_assert(L::col_dq(NBUF - 1) + (NBUF == 2 ? BM : D) <= L::TMEM_COLS, "TMEM budget");
-  static_assert(L::BYTES + 1024 <= 232448, "smem budget");
+  constexpr int BM = L::BM, QS = L::QS;
+  static_assert(L::COL_Y + 128 <= L::TMEM_COLS, "TMEM budget");
+  static_assert(L::BYTES <= L::SMEM_MAX, "smem budget");
 
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  const uint32_t pad = (1024 - (smem_u32(smem_raw) & 1023)) & 1023;
+  uint8_t* smem = smem_raw + pad;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  if (L::BYTES + pad > L::SMEM_ALLOC) {
+    // The tiles need a 1024-byte aligned base and there is no room to align it.
+    if (threadIdx.x == 0) atomicCAS(&g_status[0], 0, -2);
+    return;
+  }
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
   uint64_t* kv_full = bars;
   uint64_t* q_full = kv_full + 1;
   uint64_t* q_empty = q_full + QS;
-  uint64_t* s_full = q_empty + QS;
-  uint64_t* ds_ready = s_full + NBUF;
-  uint64_t* dq_full = ds_ready + NBUF;
-  uint64_t* dq_free = dq_full + NBUF;
-  uint64_t* ds_free = dq_free + NBUF;
-  uint64_t* mma_done = ds_free + 2;
+  uint64_t* sx_full = q_empty + QS;
+  uint64_t* dp_full = sx_full + 1;
+  uint64_t* p_ready = dp_full + 1;
+  uint64_t* ds_ready = p_ready + 1;
+  uint64_t* ds_free = ds_ready + 1;
+  uint64_t* dq_full = ds_free + 1;
+  uint64_t* dq_free = dq_full + 1;
+  uint64_t* mma_done = dq_free + 1;
   uint64_t* drain = mma_done + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
   const float* s_lse = reinterpret_cast<const float*>(smem + L::OFF_LSE);
   const float* s_dvec = reinterpret_cast<const float*>(smem + L::OFF_DVEC);
-
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
+  constexpr int kLoaderWarp = 12, kMmaWarp = 13;
 
   const int hb_count = a.H * a.B;
   const int kvb = blockIdx.x / hb_count;  // causal: the first key blocks see the most queries
@@ -203,26 +225,25 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(&q_full[s], 1);
       mbar_init(&q_empty[s], 1);
     }
-    for (int s = 0; s < NBUF; ++s) {
-      mbar_init(&s_full[s], 1);
-      mbar_init(&ds_ready[s], 128);
-      mbar_init(&dq_full[s], 1);
-      mbar_init(&dq_free[s], 128);
-    }
-    mbar_init(&ds_free[0], 1);
-    mbar_init(&ds_free[1], 1);
+    mbar_init(sx_full, 1);
+    mbar_init(dp_full, 1);
+    mbar_init(p_ready, 256);
+    mbar_init(ds_ready, 256);
+    mbar_init(ds_free, 1);
+    mbar_init(dq_full, 1);
+    mbar_init(dq_free, 128);
     mbar_init(mma_done, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 8 && lane == 0) {
+  if (warp == kLoaderWarp && lane == 0) {
     prefetch_tmap(&tmQ);
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmV);
     prefetch_tmap(&tmdO);
   }
-  if (warp == 9) {
+  if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, L::TMEM_COLS);
     tmem_relinquish();
   }
@@ -231,13 +252,13 @@ __global__ void __launch_bounds__(320, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 8) {
+  if (warp == kLoaderWarp) {
     // ---------------------------------------------------------------- loader
     if (lane == 0 && n > 0) {
-      mbar_arrive_expect_tx(kv_full, 2 * L::KV_TILE);
+      mbar_arrive_expect_tx(kv_full, 2 * L::TILE);
       for (int kb = 0; kb < L::KB; ++kb) {
-        tma_load_4d(smem + L::OFF_K + kb * L::KV_BLK, &tmK, kv_full, kb * 64, n0, h, b);
-        tma_load_4d(smem + L::OFF_V + kb * L::KV_BLK, &tmV, kv_full, kb * 64, n0, h, b);
+        tma_load_4d(smem + L::OFF_K + kb * L::BLK, &tmK, kv_full, kb * 64, n0, h, b);
+        tma_load_4d(smem + L::OFF_V + kb * L::BLK, &tmV, kv_full, kb * 64, n0, h, b);
       }
       int i = 0;
       for (; i < n; ++i) {
@@ -245,10 +266,10 @@ __global__ void __launch_bounds__(320, 1)
         const uint32_t ph = (i / QS) & 1;
         if (!wait_bar(&q_empty[st], ph ^ 1, abort_flag, kRoleLoader, i)) break;
         const int i0 = (i_start + i) * BM;
-        mbar_arrive_expect_tx(&q_full[st], 2 * L::Q_TILE + 2 * BM * 4);
+        mbar_arrive_expect_tx(&q_full[st], 2 * L::TILE + 2 * BM * 4);
         for (int kb = 0; kb < L::KB; ++kb) {
-          tma_load_4d(smem + L::OFF_Q + st * L::Q_TILE + kb * L::Q_BLK, &tmQ, &q_full[st], kb * 64, i0, h, b);
-          tma_load_4d(smem + L::OFF_DO + st * L::Q_TILE + kb * L::Q_BLK, &tmdO, &q_full[st], kb * 64, i0, h, b);
+          tma_load_4d(smem + L::OFF_Q + st * L::TILE + kb * L::BLK, &tmQ, &q_full[st], kb * 64, i0, h, b);
+          tma_load_4d(smem + L::OFF_DO + st * L::TILE + kb * L::BLK, &tmdO, &q_full[st], kb * 64, i0, h, b);
         }
         bulk_load(smem + L::OFF_LSE + st * BM * 4, a.lse2 + bh_row0 + i0, BM * 4, &q_full[st]);
         bulk_load(smem + L::OFF_DVEC + st * BM * 4, a.dvec + bh_row0 + i0, BM * 4, &q_full[st]);
@@ -258,7 +279,7 @@ __global__ void __launch_bounds__(320, 1)
         for (int j = max(0, i - QS); j < i; ++j) drain_wait(&q_full[j % QS], (j / QS) & 1);
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == kMmaWarp) {
     // ----------------------------------------------------------- MMA issuer
     if (lane == 0 && n > 0) {
       const uint32_t sK = smem_u32(smem + L::OFF_K);
@@ -266,166 +287,183 @@ __global__ void __launch_bounds__(320, 1)
       const uint32_t sQ = smem_u32(smem + L::OFF_Q);
       const uint32_t sdO = smem_u32(smem + L::OFF_DO);
       const uint32_t sDS = smem_u32(smem + L::OFF_DS);
-      // S^T = K Q^T and dP^T = V dO^T: M = 128 keys, N = BM queries, K = D.
-      const uint32_t id_s = idesc_f16(BF16, 128, BM, 0, 0);
-      // dV += P^T dO, dK += dS^T Q: M = 128 keys, N = D, K = BM (B operand MN-major).
+      // S^T = K Q^T, dP^T = V dO^T: M = 128 keys, N = 128 queries, K = D (both K-major).
+      const uint32_t id_s = idesc_f16(BF16, 128, 128, 0, 0);
+      // dV += P^T dO, dK += dS^T Q: M = 128 keys, N = D, K = 128 queries; A in TMEM, B MN-major.
       const uint32_t id_kv = idesc_f16(BF16, 128, D, 0, 1);
-      // dQ^T = K^T dS^T (D = 128): M = D, N = BM; dQ = dS K (D = 64): M = BM, N = D. Both operands MN-major.
-      const uint32_t id_q = (NBUF == 2) ? idesc_f16(BF16, 128, BM, 1, 1) : idesc_f16(BF16, 128, D, 1, 1);
-
-      auto issue_sdp = [&](int i) {
-        const int bf = i % NBUF;
-        const int st = i % QS;
-        const uint32_t qa = sQ + st * L::Q_TILE;
-        const uint32_t da = sdO + st * L::Q_TILE;
+      // D = 128: dQ^T = K^T dS^T, M = head_dim, N = 128 queries, K = 128 keys; A = K viewed
+      // MN-major, B = dS^T MN-major. D = 64: dQ = dS K, M = 128 queries, N = D; A = dS^T
+      // viewed MN-major, B = K MN-major.
+      const uint32_t id_q = L::DQ_T ? idesc_f16(BF16, 128, 128, 1, 1) : idesc_f16(BF16, 128, D, 1, 1);
+      auto issue_kt = [&](uint32_t dcol, uint32_t kv, uint32_t qa) {  // dcol = kv-tile x qa-tile^T
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t okv = (kk >> 2) * L::KV_BLK + (kk & 3) * 32;
-          const uint32_t oq = (kk >> 2) * L::Q_BLK + (kk & 3) * 32;
-          mma_ss(tmem + L::col_s(bf), desc_sw128(sK + okv, 16, 1024), desc_sw128(qa + oq, 16, 1024), id_s, kk > 0);
+          const uint32_t o = (kk >> 2) * L::BLK + (kk & 3) * 32;
+          mma_ss(tmem + dcol, desc_sw128(kv + o, 16, 1024), desc_sw128(qa + o, 16, 1024), id_s, kk > 0);
         }
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t okv = (kk >> 2) * L::KV_BLK + (kk & 3) * 32;
-          const uint32_t oq = (kk >> 2) * L::Q_BLK + (kk & 3) * 32;
-          mma_ss(tmem + L::col_dp(bf), desc_sw128(sV + okv, 16, 1024), desc_sw128(da + oq, 16, 1024), id_s, kk > 0);
-        }
-        mma_commit(&s_full[bf]);
       };
-
       bool ok = wait_bar(kv_full, 0, abort_flag, kRoleMma, -1) && wait_bar(&q_full[0], 0, abort_flag, kRoleMma, 0);
       if (ok) {
         tc_fence_after();
-        issue_sdp(0);
+        issue_kt(L::COL_X, sK, sQ);
+        mma_commit(sx_full);
+        issue_kt(L::COL_Y, sV, sdO);
+        mma_commit(dp_full);
       }
       for (int i = 0; ok && i < n; ++i) {
-        const int bf = i % NBUF;
         const int st = i % QS;
-        const int db = i & 1;
-        if (NBUF == 2 && i + 1 < n) {
-          // The other buffer held S^T/dP^T(i-1) and then dQ^T(i-1): wait until it is drained.
-          if (i >= 1 && !(ok = wait_bar(&dq_free[(i - 1) % NBUF], ((i - 1) / NBUF) & 1, abort_flag, kRoleMma, i)))
-            break;
-          if (!(ok = wait_bar(&q_full[(i + 1) % QS], ((i + 1) / QS) & 1, abort_flag, kRoleMma, i + 1))) break;
-          tc_fence_after();
-          issue_sdp(i + 1);
-        }
-        if (!(ok = wait_bar(&ds_ready[bf], (i / NBUF) & 1, abort_flag, kRoleMma, i))) break;
+        const uint32_t ph = i & 1;
+        const uint32_t qa = sQ + st * L::TILE;
+        const uint32_t da = sdO + st * L::TILE;
+        if (!(ok = wait_bar(p_ready, ph, abort_flag, kRoleMma, i))) break;
         tc_fence_after();
-        const uint32_t qa = sQ + st * L::Q_TILE;
-        const uint32_t da = sdO + st * L::Q_TILE;
-        const uint32_t dsa = sDS + db * L::DS_TILE;
-        // dV += P^T dO  (P^T in TMEM, 16-bit pairs in the S^T columns)
+        // dV += P^T dO
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk)
-          mma_ts(tmem + L::COL_DV, tmem + L::col_s(bf) + kk * 8, desc_sw128(da + kk * 2048, L::Q_BLK, 1024), id_kv,
+          mma_ts(tmem + L::COL_DV, tmem + L::col_p(kk), desc_sw128(da + kk * 2048, L::BLK, 1024), id_kv,
                  (i > 0 || kk > 0) ? 1u : 0u);
-        // dK += dS^T Q  (dS^T K-major in smem: [128 keys][BM] in 64-column blocks)
+        if (!(ok = wait_bar(ds_ready, ph, abort_flag, kRoleMma, i))) break;
+        tc_fence_after();
+        // dK += dS^T Q
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk)
-          mma_ss(tmem + L::COL_DK, desc_sw128(dsa + (kk >> 2) * L::KV_BLK + (kk & 3) * 32, 16, 1024),
-                 desc_sw128(qa + kk * 2048, L::Q_BLK, 1024), id_kv, (i > 0 || kk > 0) ? 1u : 0u);
+          mma_ts(tmem + L::COL_DK, tmem + L::col_ds(kk), desc_sw128(qa + kk * 2048, L::BLK, 1024), id_kv,
+                 (i > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&q_empty[st]);
-        if (NBUF == 1 && i >= 1)
-          if (!(ok = wait_bar(&dq_free[0], (i - 1) & 1, abort_flag, kRoleMma, i))) break;
-        if (NBUF == 2) {
-          // dQ^T = K^T dS^T: A = K viewed MN-major (M = head_dim), B = dS^T MN-major (N = queries).
-#pragma unroll
-          for (int kk = 0; kk < L::BN / 16; ++kk)
-            mma_ss(tmem + L::col_dq(bf), desc_sw128(sK + kk * 2048, L::KV_BLK, 1024),
-                   desc_sw128(dsa + kk * 2048, L::KV_BLK, 1024), id_q, kk > 0);
-        } else {
-          // dQ = dS K: A = dS^T viewed MN-major (M = queries), B = K MN-major (N = head_dim).
-#pragma unroll
-          for (int kk = 0; kk < L::BN / 16; ++kk)
-            mma_ss(tmem + L::col_dq(0), desc_sw128(dsa + kk * 2048, L::KV_BLK, 1024),
-                   desc_sw128(sK + kk * 2048, L::KV_BLK, 1024), id_q, kk > 0);
-        }
-        mma_commit(&dq_full[bf]);
-        mma_commit(&ds_free[db]);
-        if (NBUF == 1 && i + 1 < n) {
-          if (!(ok = wait_bar(&q_full[(i + 1) % QS], ((i + 1) / QS) & 1, abort_flag, kRoleMma, i + 1))) break;
+        // S^T(i+1) into X: issued after the MMAs that read P^T, dS^T from X.
+        if (i + 1 < n) {
+          const int sn = (i + 1) % QS;
+          if (!(ok = wait_bar(&q_full[sn], ((i + 1) / QS) & 1, abort_flag, kRoleMma, i + 1))) break;
           tc_fence_after();
-          issue_sdp(i + 1);
+          issue_kt(L::COL_X, sK, sQ + sn * L::TILE);
+          mma_commit(sx_full);
+        }
+        // dQ (or dQ^T) into Y: dP^T(i) there has been read by the softmax warps.
+#pragma unroll
+        for (int kk = 0; kk < L::BN / 16; ++kk) {
+          const uint64_t dk_desc = desc_sw128(sDS + kk * 2048, L::BLK, 1024);
+          const uint64_t k_desc = desc_sw128(sK + kk * 2048, L::BLK, 1024);
+          if constexpr (L::DQ_T)
+            mma_ss(tmem + L::COL_Y, k_desc, dk_desc, id_q, kk > 0);
+          else
+            mma_ss(tmem + L::COL_Y, dk_desc, k_desc, id_q, kk > 0);
+        }
+        mma_commit(dq_full);
+        mma_commit(ds_free);
+        // dP^T(i+1) into Y once dQ(i) has been read out of it.
+        if (i + 1 < n) {
+          if (!(ok = wait_bar(dq_free, ph, abort_flag, kRoleMma, i))) break;
+          tc_fence_after();
+          issue_kt(L::COL_Y, sV, sdO + ((i + 1) % QS) * L::TILE);
+          mma_commit(dp_full);
         }
       }
       mma_commit(mma_done);
       mma_commit(drain);
       drain_wait(drain, 0);
     }
-  } else if (warp < 4) {
-    // ------------------------------------------------ P^T, dS^T (one key per thread)
-    const int kr = warp * 32 + lane;
+  } else if (warp < 8) {
+    // --------------- P^T and dS^T: one key row per thread, 64 query columns per warpgroup
+    const int g = warp >> 2;
+    const int kr = (warp & 3) * 32 + lane;
     const int key = n0 + kr;
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tX = tmem + lane_base + L::COL_X + 64 * g;
+    const uint32_t tY = tmem + lane_base + L::COL_Y + 64 * g;
     const float sl2 = a.scale_log2;
     bool ok = true;
     for (int i = 0; i < n; ++i) {
-      const int bf = i % NBUF;
       const int st = i % QS;
-      const int db = i & 1;
-      ok = __all_sync(0xffffffffu, wait_bar(&s_full[bf], (i / NBUF) & 1, abort_flag, kRoleSoftmax, i) &&
-                                       wait_bar(&q_full[st], (i / QS) & 1, abort_flag, kRoleSoftmax, i) &&
-                                       wait_bar(&ds_free[db], ((i >> 1) & 1) ^ 1, abort_flag, kRoleSoftmax, i));
+      const uint32_t ph = i & 1;
+      ok = __all_sync(0xffffffffu, wait_bar(sx_full, ph, abort_flag, kRoleSoftmax, i) &&
+                                       wait_bar(&q_full[st], (i / QS) & 1, abort_flag, kRoleSoftmax, i));
       if (!ok) break;
       tc_fence_after();
       const int i0 = (i_start + i) * BM;
-      // columns c < cmin are masked for this key (causal), all columns if key >= Sk
+      // query columns c < cmin are masked for this key (causal); all of them if key >= Sk
       int cmin = a.causal ? key - off - i0 : -1;
       if (key >= a.Sk) cmin = BM;
-      const float* lse_s = s_lse + st * BM;
-      const float* dvec_s = s_dvec + st * BM;
-      const uint32_t ds_row = smem_u32(smem + L::OFF_DS + db * L::DS_TILE) + kr * 128;
-#pragma unroll
-      for (int c = 0; c < BM / 32; ++c) {
-        uint32_t sv[32], dpv[32];
-        tmem_ld32(tmem + lane_base + L::col_s(bf) + 32 * c, sv);
-        tmem_ld32(tmem + lane_base + L::col_dp(bf) + 32 * c, dpv);
+      const float* lse_s = s_lse + st * BM + 64 * g;
+      const float* dvec_s = s_dvec + st * BM + 64 * g;
+      const int cm = cmin - 64 * g;  // in this warpgroup's column numbering
+      // Phase A: P^T = 2^(S^T scale log2e - lse2) -> 16-bit pairs into X.
+      uint32_t pp[2][16];
+      {
+        uint32_t sv[2][32];
+        tmem_ld32(tX, sv[0]);
+        tmem_ld32(tX + 32, sv[1]);
         tmem_ld_wait();
-        reg_fence(sv);
+        reg_fence(sv[0]);
+        reg_fence(sv[1]);
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const int q = 32 * c + e;
+            float s0 = __uint_as_float(sv[c][e]), s1 = __uint_as_float(sv[c][e + 1]);
+            s0 = (q < cm) ? -INFINITY : s0;
+            s1 = (q + 1 < cm) ? -INFINITY : s1;
+            const float p0 = ex2(fmaf(s0, sl2, -lse_s[q]));
+            const float p1 = ex2(fmaf(s1, sl2, -lse_s[q + 1]));
+            pp[c][e >> 1] = pack2<BF16>(p0, p1);
+          }
+      }
+      tmem_st16(tX, pp[0]);       // X columns [64g, 64g + 32): read above
+      tmem_st16(tX + 16, pp[1]);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(p_ready);
+      // Phase B: dS^T = P^T (dP^T - Dvec) -> 16-bit pairs into X and into smem.
+      ok = __all_sync(0xffffffffu, wait_bar(dp_full, ph, abort_flag, kRoleSoftmax, i) &&
+                                       wait_bar(ds_free, ph ^ 1, abort_flag, kRoleSoftmax, i));
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t ds_row = smem_u32(smem + L::OFF_DS + g * L::BLK) + kr * 128;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t dpv[32];
+        tmem_ld32(tY + 32 * c, dpv);
+        tmem_ld_wait();
         reg_fence(dpv);
-        uint32_t pp[16], dsp[16];
+        uint32_t dsp[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
           const int q = 32 * c + e;
-          float s0 = __uint_as_float(sv[e]), s1 = __uint_as_float(sv[e + 1]);
-          s0 = (q < cmin) ? -INFINITY : s0;
-          s1 = (q + 1 < cmin) ? -INFINITY : s1;
-          const float p0 = ex2(fmaf(s0, sl2, -lse_s[q]));
-          const float p1 = ex2(fmaf(s1, sl2, -lse_s[q + 1]));
-          const float d0 = p0 * (__uint_as_float(dpv[e]) - dvec_s[q]);
-          const float d1 = p1 * (__uint_as_float(dpv[e + 1]) - dvec_s[q + 1]);
-          pp[e >> 1] = pack2<BF16>(p0, p1);
+          const float2 pf = unpack2<BF16>(pp[c][e >> 1]);
+          const float d0 = pf.x * (__uint_as_float(dpv[e]) - dvec_s[q]);
+          const float d1 = pf.y * (__uint_as_float(dpv[e + 1]) - dvec_s[q + 1]);
           dsp[e >> 1] = pack2<BF16>(d0, d1);
         }
-        tmem_st16(tmem + lane_base + L::col_s(bf) + 16 * c, pp);
-        // dS^T row kr, query columns [32c, 32c + 32): four 16-byte chunks,
-        // 128-byte swizzle within each 64-column block.
+        tmem_st16(tX + 32 + 16 * c, dsp);  // X columns [64g + 32, 64g + 64): read in phase A
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          const int chunk = 4 * (c & 1) + u;
-          const uint32_t addr = ds_row + (c >> 1) * L::KV_BLK + ((chunk ^ (kr & 7)) << 4);
-          st_shared_v4(addr, dsp[4 * u], dsp[4 * u + 1], dsp[4 * u + 2], dsp[4 * u + 3]);
+          const int chunk = 4 * c + u;
+          st_shared_v4(ds_row + ((chunk ^ (kr & 7)) << 4), dsp[4 * u], dsp[4 * u + 1], dsp[4 * u + 2],
+                       dsp[4 * u + 3]);
         }
       }
       tmem_st_wait();
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(&ds_ready[bf]);
+      mbar_arrive(ds_ready);
     }
-    // epilogue: dK = scale * accumulator
+    // epilogue: warpgroup 0 writes dK = scale * accumulator, warpgroup 1 writes dV
     const bool have = n > 0;
     if (ok && !*abort_flag) {
       bool done = !have || __all_sync(0xffffffffu, wait_bar(mma_done, 0, abort_flag, kRoleSoftmax, n));
       if (done) {
         tc_fence_after();
-        uint16_t* dst = reinterpret_cast<uint16_t*>(a.dk) + b * a.dk_sb + static_cast<int64_t>(key) * a.dk_ss +
-                        h * a.dk_sh;
-#pragma unroll 1
+        const float mul = g == 0 ? a.scale : 1.f;
+        uint16_t* dst = g == 0 ? reinterpret_cast<uint16_t*>(a.dk) + b * a.dk_sb +
+                                     static_cast<int64_t>(key) * a.dk_ss + h * a.dk_sh
+                               : reinterpret_cast<uint16_t*>(a.dv) + b * a.dv_sb +
+                                     static_cast<int64_t>(key) * a.dv_ss + h * a.dv_sh;
+        const int col = g == 0 ? L::COL_DK : L::COL_DV;
+#pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t v[32];
           if (have) {
-            tmem_ld32(tmem + lane_base + L::COL_DK + 32 * c, v);
+            tmem_ld32(tmem + lane_base + col + 32 * c, v);
             tmem_ld_wait();
             reg_fence(v);
           } else {
@@ -439,8 +477,8 @@ __global__ void __launch_bounds__(320, 1)
               uint32_t w[4];
 #pragma unroll
               for (int e = 0; e < 4; ++e)
-                w[e] = pack2<BF16>(__uint_as_float(v[8 * u + 2 * e]) * a.scale,
-                                   __uint_as_float(v[8 * u + 2 * e + 1]) * a.scale);
+                w[e] = pack2<BF16>(__uint_as_float(v[8 * u + 2 * e]) * mul,
+                                   __uint_as_float(v[8 * u + 2 * e + 1]) * mul);
               d4[u] = make_uint4(w[0], w[1], w[2], w[3]);
             }
           }
@@ -448,84 +486,48 @@ __global__ void __launch_bounds__(320, 1)
       }
     }
   } else {
-    // ------------------------------------------- dQ drain (warps 4-7), then dV
-    const int wq = warp - 4;
-    const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
-    const int tr = wq * 32 + lane;  // TMEM lane: head_dim index (D = 128) or query row (D = 64)
-    bool ok = true;
+    // ------------------------------------------------- dQ drain (warps 8-11)
+    const int tr = (warp & 3) * 32 + lane;  // TMEM lane
+    const uint32_t tY = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16) + L::COL_Y;
     for (int i = 0; i < n; ++i) {
-      const int bf = i % NBUF;
-      ok = __all_sync(0xffffffffu, wait_bar(&dq_full[bf], (i / NBUF) & 1, abort_flag, kRoleSoftmax, i));
+      const bool ok = __all_sync(0xffffffffu, wait_bar(dq_full, i & 1, abort_flag, kRoleSoftmax, i));
       if (!ok) break;
       tc_fence_after();
-      const int i0 = (i_start + i) * BM;
-      if constexpr (NBUF == 2) {
-        // dQ^T: lane = head_dim index d, columns = BM = 64 query rows.
-        uint32_t v0[32], v1[32];
-        tmem_ld32(tmem + lane_base + L::col_dq(bf), v0);
-        tmem_ld32(tmem + lane_base + L::col_dq(bf) + 32, v1);
-        tmem_ld_wait();
-        reg_fence(v0);
-        reg_fence(v1);
-        tc_fence_before();
-        mbar_arrive(&dq_free[bf]);
-        float* base = a.dq_acc + (bh_row0 + i0) * D + tr;
+      const int64_t row0 = bh_row0 + (i_start + i) * BM;
+      if constexpr (L::DQ_T) {
+        // lane = head_dim index d, columns = 128 query rows: for each query the
+        // warp adds 32 consecutive floats (one 128-byte line).
+        float* col = a.dq_acc + row0 * D + tr;
 #pragma unroll
-        for (int c = 0; c < 32; ++c) red_add_f32(base + c * D, __uint_as_float(v0[c]));
-#pragma unroll
-        for (int c = 0; c < 32; ++c) red_add_f32(base + (32 + c) * D, __uint_as_float(v1[c]));
-      } else {
-        // dQ: lane = query row, columns = head_dim (64).
-        uint32_t v0[32], v1[32];
-        tmem_ld32(tmem + lane_base + L::col_dq(0), v0);
-        tmem_ld32(tmem + lane_base + L::col_dq(0) + 32, v1);
-        tmem_ld_wait();
-        reg_fence(v0);
-        reg_fence(v1);
-        tc_fence_before();
-        mbar_arrive(&dq_free[0]);
-        float* base = a.dq_acc + (bh_row0 + i0 + tr) * D;
-#pragma unroll
-        for (int c = 0; c < 32; c += 4)
-          red_add_v4_f32(base + c, __uint_as_float(v0[c]), __uint_as_float(v0[c + 1]), __uint_as_float(v0[c + 2]),
-                         __uint_as_float(v0[c + 3]));
-#pragma unroll
-        for (int c = 0; c < 32; c += 4)
-          red_add_v4_f32(base + 32 + c, __uint_as_float(v1[c]), __uint_as_float(v1[c + 1]),
-                         __uint_as_float(v1[c + 2]), __uint_as_float(v1[c + 3]));
-      }
-    }
-    // epilogue: dV
-    const int key = n0 + tr;
-    const bool have = n > 0;
-    if (ok && !*abort_flag) {
-      bool done = !have || __all_sync(0xffffffffu, wait_bar(mma_done, 0, abort_flag, kRoleSoftmax, n));
-      if (done) {
-        tc_fence_after();
-        uint16_t* dst = reinterpret_cast<uint16_t*>(a.dv) + b * a.dv_sb + static_cast<int64_t>(key) * a.dv_ss +
-                        h * a.dv_sh;
-#pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
+        for (int part = 0; part < 4; ++part) {
           uint32_t v[32];
-          if (have) {
-            tmem_ld32(tmem + lane_base + L::COL_DV + 32 * c, v);
-            tmem_ld_wait();
-            reg_fence(v);
-          } else {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = 0u;
+          tmem_ld32(tY + 32 * part, v);
+          tmem_ld_wait();
+          reg_fence(v);
+          if (part == 3) {
+            tc_fence_before();
+            mbar_arrive(dq_free);  // Y may take dP^T(i+1) now
           }
-          if (key < a.Sk) {
-            uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              uint32_t w[4];
+          for (int c = 0; c < 32; ++c) red_add_f32(col + (32 * part + c) * D, __uint_as_float(v[c]));
+        }
+      } else {
+        // lane = query row, columns = head_dim (64).
+        float* row = a.dq_acc + (row0 + tr) * D;
 #pragma unroll
-              for (int e = 0; e < 4; ++e)
-                w[e] = pack2<BF16>(__uint_as_float(v[8 * u + 2 * e]), __uint_as_float(v[8 * u + 2 * e + 1]));
-              d4[u] = make_uint4(w[0], w[1], w[2], w[3]);
-            }
+        for (int part = 0; part < D / 32; ++part) {
+          uint32_t v[32];
+          tmem_ld32(tY + 32 * part, v);
+          tmem_ld_wait();
+          reg_fence(v);
+          if (part == D / 32 - 1) {
+            tc_fence_before();
+            mbar_arrive(dq_free);
           }
+#pragma unroll
+          for (int c = 0; c < 32; c += 4)
+            red_add_v4_f32(row + 32 * part + c, __uint_as_float(v[c]), __uint_as_float(v[c + 1]),
+                           __uint_as_float(v[c + 2]), __uint_as_float(v[c + 3]));
         }
       }
     }
@@ -533,7 +535,7 @@ __global__ void __launch_bounds__(320, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == kMmaWarp) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, L::TMEM_COLS);

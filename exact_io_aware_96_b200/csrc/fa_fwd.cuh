@@ -276,14 +276,17 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
         for (int i = 0; i < 128; ++i) x[i] = (i <= lim) ? x[i] : -INFINITY;
       }
-      float mx0 = x[0], mx1 = x[1], mx2 = x[2], mx3 = x[3];
+      float mx0 = max3(x[0], x[1], x[2]), mx1 = max3(x[3], x[4], x[5]);
+      float mx2 = max3(x[6], x[7], x[8]), mx3 = max3(x[9], x[10], x[11]);
 #pragma unroll
-      for (int i = 4; i < 128; i += 4) {
-        mx0 = fmaxf(mx0, x[i]);
-        mx1 = fmaxf(mx1, x[i + 1]);
-        mx2 = fmaxf(mx2, x[i + 2]);
-        mx3 = fmaxf(mx3, x[i + 3]);
+      for (int i = 12; i < 124; i += 8) {
+        mx0 = max3(mx0, x[i], x[i + 1]);
+        mx1 = max3(mx1, x[i + 2], x[i + 3]);
+        mx2 = max3(mx2, x[i + 4], x[i + 5]);
+        mx3 = max3(mx3, x[i + 6], x[i + 7]);
       }
+      mx0 = max3(mx0, x[124], x[125]);
+      mx1 = max3(mx1, x[126], x[127]);
       const float m_blk = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
       const bool raise = m_blk > m + 8.0f;
       float alpha = 1.f;
@@ -306,24 +309,42 @@ __global__ void __launch_bounds__(320, 1)
         }
       }
       const float mu = (m == -INFINITY) ? 0.f : m;
-      float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-      uint32_t p[2][32];
+      // P = 2^(s * scale * log2e - m) for pairs of columns; one pair in four
+      // takes the polynomial exp2 on the FMA pipe, the rest the MUFU unit.
+      const uint64_t sl2x2 = f2(sl2, sl2);
+      const uint64_t negmu2 = f2(-mu, -mu);
+      uint64_t acc0 = f2(0.f, 0.f), acc1 = f2(0.f, 0.f);
 #pragma unroll
-      for (int i = 0; i < 64; i += 2) {
-        const float e0 = ex2(fmaf(x[2 * i + 0], sl2, -mu));
-        const float e1 = ex2(fmaf(x[2 * i + 1], sl2, -mu));
-        const float e2 = ex2(fmaf(x[2 * i + 2], sl2, -mu));
-        const float e3 = ex2(fmaf(x[2 * i + 3], sl2, -mu));
-        s0 += e0;
-        s1 += e1;
-        s2 += e2;
-        s3 += e3;
-        p[i >> 5][i & 31] = pack2<BF16>(e0, e1);
-        p[(i + 1) >> 5][(i + 1) & 31] = pack2<BF16>(e2, e3);
+      for (int q = 0; q < 4; ++q) {  // 32 columns at a time -> 16 packed P words
+        uint32_t pw[16];
+#pragma unroll
+        for (int cc = 0; cc < 16; ++cc) {
+          const int c = 16 * q + cc;
+          const uint64_t tt = fma2(f2(x[2 * c], x[2 * c + 1]), sl2x2, negmu2);
+          uint64_t e;
+          if ((c & 3) == 3) {
+            e = exp2_poly2(tt);
+          } else {
+            float t0, t1;
+            f2_split(tt, t0, t1);
+            e = f2(ex2(t0), ex2(t1));
+          }
+          if (c & 1)
+            acc1 = add2(acc1, e);
+          else
+            acc0 = add2(acc0, e);
+          float e0, e1;
+          f2_split(e, e0, e1);
+          pw[cc] = pack2<BF16>(e0, e1);
+        }
+        tmem_st16(tS + 16 * q, pw);  // S columns [0, 64) were read already
       }
-      l += (s0 + s1) + (s2 + s3);
-      tmem_st32(tS, p[0]);
-      tmem_st32(tS + 32, p[1]);
+      {
+        const uint64_t acc = add2(acc0, acc1);
+        float a0, a1;
+        f2_split(acc, a0, a1);
+        l += a0 + a1;
+      }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&p_full[t]);
@@ -332,7 +353,7 @@ __global__ void __launch_bounds__(320, 1)
     // Epilogue: O = O_t / l, LSE = ln2 * (m + log2 l).
     if (ok && !*abort_flag && r0 < a.Sq) {
       const bool valid = row < a.Sq;
-      const bool has = l > 0.f;
+      const bool has = (m != -INFINITY) && l > 0.f;  // m stays -inf only for rows with no allowed key
       const float inv_l = has ? 1.f / l : 0.f;
       uint16_t* orow = reinterpret_cast<uint16_t*>(a.o) + static_cast<int64_t>(b) * a.o_sb +
                        static_cast<int64_t>(row) * a.o_ss + static_cast<int64_t>(h) * a.o_sh;

@@ -161,6 +161,26 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
+// Bulk reduce-add of `bytes` fp32 values from CTA shared memory into global
+// memory (element-wise atomic adds at L2), tracked as one bulk group.
+__device__ __forceinline__ void bulk_reduce_add_f32(float* dst, const void* src, uint32_t bytes) {
+  asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(
+                   reinterpret_cast<uint64_t>(dst)),
+               "r"(smem_u32(src)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until the source reads of every committed bulk group have finished.
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// Wait until every committed bulk group has completed.
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// Barrier among `count` threads (a multiple of 32) on hardware barrier `id` (1..15).
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+__device__ __forceinline__ void st_shared_f32(uint32_t addr, float v) {
+  asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
 __device__ __forceinline__ void red_add_f32(float* addr, float v) {
   asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(v) : "memory");
 }
@@ -237,6 +257,60 @@ __device__ __forceinline__ float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// ------------------------------------------------------ packed fp32 pairs
+// Two fp32 values in one 64-bit register, `lo` in the low half; sm_100 runs
+// fma/add on such pairs as one instruction (f32x2).
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_split(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^t for a pair, on the FMA and integer pipes instead of the MUFU unit.
+// Cody-Waite range reduction t = n + f, n = rint(t), f in [-1/2, 1/2]; then
+// 2^f from a degree-3 polynomial fitted for minimum maximum relative error on
+// [-1/2, 1/2] (fit_exp2_poly.py beside this file; max relative error 7.5e-5),
+// and 2^n added into the exponent field. t is clamped below at -126, so
+// arguments under it (including -inf) give a value below 2^-125, not 0:
+// callers that need exact zeros must not rely on this path for them.
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t t) {
+  constexpr float kMagic = 12582912.f;  // 1.5 * 2^23: adding it rounds to an integer in the low mantissa bits
+  float t0, t1;
+  f2_split(t, t0, t1);
+  t = f2(fmaxf(t0, -126.f), fmaxf(t1, -126.f));
+  const uint64_t r = add2(t, f2(kMagic, kMagic));
+  const uint64_t n = add2(r, f2(-kMagic, -kMagic));
+  const uint64_t f = fma2(n, f2(-1.f, -1.f), t);
+  uint64_t p = fma2(f2(0.0551716685f, 0.0551716685f), f, f2(0.242611125f, 0.242611125f));
+  p = fma2(p, f, f2(0.693260968f, 0.693260968f));
+  p = fma2(p, f, f2(0.999928057f, 0.999928057f));
+  float p0, p1, r0, r1;
+  f2_split(p, p0, p1);
+  f2_split(r, r0, r1);
+  // low bits of r hold n (the magic constant's own bits vanish under << 23)
+  const uint32_t e0 = __float_as_uint(p0) + (__float_as_uint(r0) << 23);
+  const uint32_t e1 = __float_as_uint(p1) + (__float_as_uint(r1) << 23);
+  return f2(__uint_as_float(e0), __uint_as_float(e1));
+}
+
 // Two floats -> packed 16-bit pair, `lo` in the low half. Round to nearest even.
 template <bool BF16>
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
