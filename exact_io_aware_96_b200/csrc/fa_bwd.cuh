@@ -35,9 +35,9 @@
 // X (S^T, then 16-bit P^T and dS^T written back by the softmax warps and used
 // as the TMEM A operand of dV += P^T dO and dK += dS^T Q) and Y (dP^T, then
 // dQ^T = K^T dS^T (D = 128) or dQ = dS K (D = 64), with dS^T staged in
-// 128-byte swizzled smem). The
-// MMA order per block i is dV(i), dK(i), S^T(i+1), dQ(i), dP^T(i+1), so the
-// softmax of block i+1 starts while dQ(i) and dP^T(i+1) run.
+// 128-byte swizzled smem). The MMA order per block i is dV(i), dK(i), dQ(i),
+// S^T(i+1), dP^T(i+1): S^T(i+1) runs while dQ(i) is drained out of Y, and the
+// softmax of block i+1 starts while dP^T(i+1) runs.
 //
 // Page legend: [P1] "Miniconda-Python3.9环境下使用FlashAttention优化训练";
 // [P2] "使用FlashAttention优化PyTorch模型注意力计算"; [P4] the FlashAttention-2
@@ -330,14 +330,6 @@ __global__ void __launch_bounds__(448, 1)
           mma_ts(tmem + L::COL_DK, tmem + L::col_ds(kk), desc_sw128(qa + kk * 2048, L::BLK, 1024), id_kv,
                  (i > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&q_empty[st]);
-        // S^T(i+1) into X: issued after the MMAs that read P^T, dS^T from X.
-        if (i + 1 < n) {
-          const int sn = (i + 1) % QS;
-          if (!(ok = wait_bar(&q_full[sn], ((i + 1) / QS) & 1, abort_flag, kRoleMma, i + 1))) break;
-          tc_fence_after();
-          issue_kt(L::COL_X, sK, sQ + sn * L::TILE);
-          mma_commit(sx_full);
-        }
         // dQ (or dQ^T) into Y: dP^T(i) there has been read by the softmax warps.
 #pragma unroll
         for (int kk = 0; kk < L::BN / 16; ++kk) {
@@ -350,11 +342,18 @@ __global__ void __launch_bounds__(448, 1)
         }
         mma_commit(dq_full);
         mma_commit(ds_free);
-        // dP^T(i+1) into Y once dQ(i) has been read out of it.
         if (i + 1 < n) {
+          // S^T(i+1) into X (after the MMAs that read P^T, dS^T from X); it
+          // runs while the dQ block is drained out of Y.
+          const int sn = (i + 1) % QS;
+          if (!(ok = wait_bar(&q_full[sn], ((i + 1) / QS) & 1, abort_flag, kRoleMma, i + 1))) break;
+          tc_fence_after();
+          issue_kt(L::COL_X, sK, sQ + sn * L::TILE);
+          mma_commit(sx_full);
+          // dP^T(i+1) into Y once dQ(i) has been read out of it.
           if (!(ok = wait_bar(dq_free, ph, abort_flag, kRoleMma, i))) break;
           tc_fence_after();
-          issue_kt(L::COL_Y, sV, sdO + ((i + 1) % QS) * L::TILE);
+          issue_kt(L::COL_Y, sV, sdO + sn * L::TILE);
           mma_commit(dp_full);
         }
       }
