@@ -391,20 +391,26 @@ __global__ void __launch_bounds__(448, 1)
         uint32_t sv[2][32];
         tmem_ld32(tX, sv[0]);
         tmem_ld32(tX + 32, sv[1]);
+        float4 lv[16];  // lse2 of this warpgroup's 64 queries, loaded while the TMEM load is in flight
+#pragma unroll
+        for (int u = 0; u < 16; ++u) lv[u] = reinterpret_cast<const float4*>(lse_s)[u];
         tmem_ld_wait();
         reg_fence(sv[0]);
         reg_fence(sv[1]);
 #pragma unroll
         for (int c = 0; c < 2; ++c)
 #pragma unroll
-          for (int e = 0; e < 32; e += 2) {
+          for (int e = 0; e < 32; e += 4) {
             const int q = 32 * c + e;
+            const float4 L4 = lv[q >> 2];
             float s0 = __uint_as_float(sv[c][e]), s1 = __uint_as_float(sv[c][e + 1]);
+            float s2 = __uint_as_float(sv[c][e + 2]), s3 = __uint_as_float(sv[c][e + 3]);
             s0 = (q < cm) ? -INFINITY : s0;
             s1 = (q + 1 < cm) ? -INFINITY : s1;
-            const float p0 = ex2(fmaf(s0, sl2, -lse_s[q]));
-            const float p1 = ex2(fmaf(s1, sl2, -lse_s[q + 1]));
-            pp[c][e >> 1] = pack2<BF16>(p0, p1);
+            s2 = (q + 2 < cm) ? -INFINITY : s2;
+            s3 = (q + 3 < cm) ? -INFINITY : s3;
+            pp[c][e >> 1] = pack2<BF16>(ex2(fmaf(s0, sl2, -L4.x)), ex2(fmaf(s1, sl2, -L4.y)));
+            pp[c][(e >> 1) + 1] = pack2<BF16>(ex2(fmaf(s2, sl2, -L4.z)), ex2(fmaf(s3, sl2, -L4.w)));
           }
       }
       tmem_st16(tX, pp[0]);       // X columns [64g, 64g + 32): read above
@@ -422,16 +428,20 @@ __global__ void __launch_bounds__(448, 1)
       for (int c = 0; c < 2; ++c) {
         uint32_t dpv[32];
         tmem_ld32(tY + 32 * c, dpv);
+        float4 dv4[8];  // Dvec of these 32 queries, loaded while the TMEM load is in flight
+#pragma unroll
+        for (int u = 0; u < 8; ++u) dv4[u] = reinterpret_cast<const float4*>(dvec_s + 32 * c)[u];
         tmem_ld_wait();
         reg_fence(dpv);
         uint32_t dsp[16];
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const int q = 32 * c + e;
-          const float2 pf = unpack2<BF16>(pp[c][e >> 1]);
-          const float d0 = pf.x * (__uint_as_float(dpv[e]) - dvec_s[q]);
-          const float d1 = pf.y * (__uint_as_float(dpv[e + 1]) - dvec_s[q + 1]);
-          dsp[e >> 1] = pack2<BF16>(d0, d1);
+        for (int e = 0; e < 32; e += 4) {
+          const float4 V4 = dv4[e >> 2];
+          const float2 pa = unpack2<BF16>(pp[c][e >> 1]);
+          const float2 pb = unpack2<BF16>(pp[c][(e >> 1) + 1]);
+          dsp[e >> 1] = pack2<BF16>(pa.x * (__uint_as_float(dpv[e]) - V4.x), pa.y * (__uint_as_float(dpv[e + 1]) - V4.y));
+          dsp[(e >> 1) + 1] =
+              pack2<BF16>(pb.x * (__uint_as_float(dpv[e + 2]) - V4.z), pb.y * (__uint_as_float(dpv[e + 3]) - V4.w));
         }
         tmem_st16(tX + 32 + 16 * c, dsp);  // X columns [64g + 32, 64g + 64): read in phase A
 #pragma unroll

@@ -39,9 +39,7 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatil
   if (sm100::mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = sm100::globaltimer_ns();
   while (true) {
-#pragma unroll 1
-    for (int i = 0; i < 32; ++i)
-      if (sm100::mbar_try_wait(bar, parity)) return true;
+    if (sm100::mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
     if (sm100::globaltimer_ns() - t0 > kWaitLimitNs) {
       *abort_flag = 1;
