@@ -47,7 +47,7 @@ int check_common(int B, int H, int Sq, int Sk, int D, float scale, int causal, i
   if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
   if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_UNSUPPORTED;
-  if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
+  if (D < 8 || D > 128 || D % 8) return FA_ERR_UNSUPPORTED;
   const int64_t lim = (int64_t(1) << 31) - 1;
   if (int64_t(B) * H * Sq > lim || int64_t(B) * H * Sk > lim) return FA_ERR_INVALID_ARG;
   if (int64_t(B) * H * ((Sq + 255) / 256) > lim) return FA_ERR_INVALID_ARG;
@@ -105,9 +105,9 @@ int launch_fwd(const fa_fwd_params* p, cudaStream_t stream) {
   int st = prepare(kern, L::SMEM_ALLOC, done);
   if (st != FA_OK) return st;
   CUtensorMap mq, mk, mv;
-  if ((st = make_map(&mq, p->q, p->B, p->Sq, p->H, D, p->dtype, 128)) != FA_OK) return st;
-  if ((st = make_map(&mk, p->k, p->B, p->Sk, p->H, D, p->dtype, 128)) != FA_OK) return st;
-  if ((st = make_map(&mv, p->v, p->B, p->Sk, p->H, D, p->dtype, 128)) != FA_OK) return st;
+  if ((st = make_map(&mq, p->q, p->B, p->Sq, p->H, p->D, p->dtype, 128)) != FA_OK) return st;
+  if ((st = make_map(&mk, p->k, p->B, p->Sk, p->H, p->D, p->dtype, 128)) != FA_OK) return st;
+  if ((st = make_map(&mv, p->v, p->B, p->Sk, p->H, p->D, p->dtype, 128)) != FA_OK) return st;
   fa::FwdArgs a;
   a.o = p->o.ptr;
   a.lse = p->lse;
@@ -121,6 +121,7 @@ int launch_fwd(const fa_fwd_params* p, cudaStream_t stream) {
   a.scale_log2 = p->scale * 1.4426950408889634f;
   a.causal = p->causal;
   a.n_qblocks = (p->Sq + 255) / 256;
+  a.d = p->D;
   const unsigned grid = unsigned(int64_t(a.n_qblocks) * p->B * p->H);
   kern<<<grid, L::kThreads, L::SMEM_ALLOC, stream>>>(mq, mk, mv, a);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
@@ -134,11 +135,11 @@ int launch_bwd(const fa_bwd_params* p, cudaStream_t stream) {
   int st = prepare(kern, L::SMEM_ALLOC, done);
   if (st != FA_OK) return st;
   CUtensorMap mq, mk, mv, mdo;
-  if ((st = make_map(&mq, p->q, p->B, p->Sq, p->H, D, p->dtype, L::BM)) != FA_OK) return st;
-  if ((st = make_map(&mk, p->k, p->B, p->Sk, p->H, D, p->dtype, L::BN)) != FA_OK) return st;
-  if ((st = make_map(&mv, p->v, p->B, p->Sk, p->H, D, p->dtype, L::BN)) != FA_OK) return st;
+  if ((st = make_map(&mq, p->q, p->B, p->Sq, p->H, p->D, p->dtype, L::BM)) != FA_OK) return st;
+  if ((st = make_map(&mk, p->k, p->B, p->Sk, p->H, p->D, p->dtype, L::BN)) != FA_OK) return st;
+  if ((st = make_map(&mv, p->v, p->B, p->Sk, p->H, p->D, p->dtype, L::BN)) != FA_OK) return st;
   static_assert(L::BM == 128 && L::BN == 128, "tensor maps assume 128-row boxes");
-  if ((st = make_map(&mdo, p->dO, p->B, p->Sq, p->H, D, p->dtype, L::BM)) != FA_OK) return st;
+  if ((st = make_map(&mdo, p->dO, p->B, p->Sq, p->H, p->D, p->dtype, L::BM)) != FA_OK) return st;
   fa::BwdArgs a;
   std::memset(&a, 0, sizeof(a));
   a.o = p->o.ptr;
@@ -164,6 +165,7 @@ int launch_bwd(const fa_bwd_params* p, cudaStream_t stream) {
   a.scale = p->scale;
   a.scale_log2 = p->scale * 1.4426950408889634f;
   a.causal = p->causal;
+  a.d = p->D;
   constexpr int G = D / 8;
   const int64_t pre_threads = rows * G;
   fa::fa_bwd_pre<D, BF16><<<unsigned((pre_threads + 255) / 256), 256, 0, stream>>>(a);
@@ -215,7 +217,7 @@ const char* fa_strerror(int s) {
   switch (s) {
     case FA_OK: return "ok";
     case FA_ERR_INVALID_ARG: return "invalid argument (null pointer, size < 1, scale or causal flag)";
-    case FA_ERR_UNSUPPORTED: return "unsupported dtype or head_dim (fp16/bf16, D in {64,128})";
+    case FA_ERR_UNSUPPORTED: return "unsupported dtype or head_dim (fp16/bf16; D a multiple of 8 in [8, 128])";
     case FA_ERR_MISALIGNED: return "tensor base or stride not 16-byte aligned";
     case FA_ERR_CUDA: return "CUDA runtime or driver call failed";
     case FA_ERR_TIMEOUT: return "device-side pipeline wait exceeded its time limit";
@@ -236,7 +238,9 @@ int fa_fwd_ex(const fa_fwd_params* p, fa_stream_t stream) {
   if (p->lse == nullptr) return FA_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(p->lse) & 3u) return FA_ERR_MISALIGNED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (p->D == 64) return p->dtype == FA_BF16 ? launch_fwd<64, true>(p, s) : launch_fwd<64, false>(p, s);
+  // head_dim <= 64 runs the 64-column kernels, <= 128 the 128-column ones;
+  // the tensor maps read the columns past head_dim as zeros.
+  if (p->D <= 64) return p->dtype == FA_BF16 ? launch_fwd<64, true>(p, s) : launch_fwd<64, false>(p, s);
   return p->dtype == FA_BF16 ? launch_fwd<128, true>(p, s) : launch_fwd<128, false>(p, s);
 }
 
@@ -262,8 +266,9 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
 
 size_t fa_bwd_workspace_size(int B, int H, int Sq, int D) {
   if (B < 1 || H < 1 || Sq < 1 || D < 1) return 0;
+  const uint64_t dpad = D <= 64 ? 64 : (D <= 128 ? 128 : uint64_t(D));  // kernel width
   const uint64_t rows = uint64_t(B) * H * ((uint64_t(Sq) + 127) / 128 * 128);
-  const uint64_t bytes = rows * (uint64_t(D) + 2) * 4;  // dq accumulator, Dvec, LSE * log2(e)
+  const uint64_t bytes = rows * (dpad + 2) * 4;  // dq accumulator, Dvec, LSE * log2(e)
   if (bytes > (uint64_t(1) << 50)) return 0;
   return size_t(bytes);
 }
@@ -281,7 +286,7 @@ int fa_bwd_ex(const fa_bwd_params* p, fa_stream_t stream) {
   if (p->workspace == nullptr || p->workspace_bytes < need || need == 0) return FA_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(p->workspace) & 255u) return FA_ERR_MISALIGNED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (p->D == 64) return p->dtype == FA_BF16 ? launch_bwd<64, true>(p, s) : launch_bwd<64, false>(p, s);
+  if (p->D <= 64) return p->dtype == FA_BF16 ? launch_bwd<64, true>(p, s) : launch_bwd<64, false>(p, s);
   return p->dtype == FA_BF16 ? launch_bwd<128, true>(p, s) : launch_bwd<128, false>(p, s);
 }
 

@@ -64,7 +64,7 @@ __global__ void __launch_bounds__(256) fa_bwd_pre(const BwdArgs a) {
   const int h = bh % a.H;
   const int b = bh / a.H;
   float acc = 0.f;
-  if (i < a.Sq) {
+  if (i < a.Sq && part * 8 < a.d) {
     const uint4 ov = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(a.o) + b * a.o_sb +
                                                       static_cast<int64_t>(i) * a.o_ss + h * a.o_sh + part * 8);
     const uint4 dv = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(a.dO) + b * a.do_sb +
@@ -102,7 +102,7 @@ __global__ void __launch_bounds__(256) fa_bwd_dq(const BwdArgs a) {
   const int64_t gid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t row = gid / G;  // (b, h, i) with i < Sq
   const int part = static_cast<int>(gid % G);
-  if (row >= static_cast<int64_t>(a.B) * a.H * a.Sq) return;
+  if (row >= static_cast<int64_t>(a.B) * a.H * a.Sq || part * 8 >= a.d) return;
   const int i = static_cast<int>(row % a.Sq);
   const int bh = static_cast<int>(row / a.Sq);
   const int h = bh % a.H;
@@ -468,8 +468,8 @@ __global__ void __launch_bounds__(448, 1)
                                : reinterpret_cast<uint16_t*>(a.dv) + b * a.dv_sb +
                                      static_cast<int64_t>(key) * a.dv_ss + h * a.dv_sh;
         const int col = g == 0 ? L::COL_DK : L::COL_DV;
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+#pragma unroll 1
+        for (int c = 0; c < (a.d + 31) / 32; ++c) {
           uint32_t v[32];
           if (have) {
             tmem_ld32(tmem + lane_base + col + 32 * c, v);
@@ -488,7 +488,7 @@ __global__ void __launch_bounds__(448, 1)
               for (int e = 0; e < 4; ++e)
                 w[e] = pack2<BF16>(__uint_as_float(v[8 * u + 2 * e]) * mul,
                                    __uint_as_float(v[8 * u + 2 * e + 1]) * mul);
-              d4[u] = make_uint4(w[0], w[1], w[2], w[3]);
+              if (32 * c + 8 * u < a.d) d4[u] = make_uint4(w[0], w[1], w[2], w[3]);
             }
           }
         }

@@ -63,6 +63,7 @@ struct FwdArgs {
   float* lse;
   int64_t o_sb, o_ss, o_sh;  // element strides of o
   int B, H, Sq, Sk;
+  int d;             // head_dim of the tensors (<= the kernel's padded D; columns past it read as 0)
   float scale_log2;  // scale * log2(e)
   int causal;
   int n_qblocks;     // ceil(Sq / 256)
@@ -84,6 +85,7 @@ struct BwdArgs {
   int64_t dk_sb, dk_ss, dk_sh;
   int64_t dv_sb, dv_ss, dv_sh;
   int B, H, Sq, Sk, Sq_pad;
+  int d;  // head_dim of the tensors (<= the kernel's padded D)
   float scale;
   float scale_log2;
   int causal;

@@ -361,7 +361,7 @@ __global__ void __launch_bounds__(320, 1)
         if (__all_sync(0xffffffffu, wait_bar(&o_final[t], 0, abort_flag, kRoleSoftmax, n))) {
           tc_fence_after();
 #pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
+          for (int c = 0; c < (a.d + 31) / 32; ++c) {
             uint32_t ov[32];
             tmem_ld32(tO + 32 * c, ov);
             tmem_ld_wait();
@@ -373,13 +373,14 @@ __global__ void __launch_bounds__(320, 1)
             if (valid) {
               uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
 #pragma unroll
-              for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+              for (int i = 0; i < 4; ++i)
+                if (32 * c + 8 * i < a.d) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
             }
           }
         }
       } else if (valid) {
         uint4* dst = reinterpret_cast<uint4*>(orow);
-        for (int i = 0; i < D / 8; ++i) dst[i] = make_uint4(0, 0, 0, 0);
+        for (int i = 0; i < a.d / 8; ++i) dst[i] = make_uint4(0, 0, 0, 0);
       }
       if (valid)
         a.lse[(static_cast<int64_t>(b) * a.H + h) * a.Sq + row] =

@@ -15,6 +15,7 @@
  *   [P2] "使用FlashAttention优化PyTorch模型注意力计算", section
  *        "FlashAttention 是如何做到又快又省内存的？" items 1-3 (fusion, tiling
  *        with an online softmax, recomputation).
+ *        Section "工程实践中的关键考量" (head_dim <= 128).
  *   [P4] the FlashAttention-2 walkthrough titled "企业官网建设流程全解析",
  *        §3.1 (unscaled output, one final rescale, only the logsumexp saved),
  *        §3.2 (parallelism over batch x heads x sequence blocks), §3.3 (five
@@ -37,7 +38,10 @@
  *   j <= i + (Sk - Sq). With Sq == Sk this is the lower triangle.
  * dtype. FA_FP16 or FA_BF16 for every tensor of a call except lse and the
  *   workspace (fp32). Anything else is FA_ERR_UNSUPPORTED ([P4] §5).
- * head_dim. D in {64, 128}; other values are FA_ERR_UNSUPPORTED.
+ * head_dim. D a multiple of 8 in [8, 128] ([P2] "工程实践中的关键考量": head_dim
+ *   <= 128); other values are FA_ERR_UNSUPPORTED. D <= 64 runs the 64-column
+ *   kernels and 64 < D <= 128 the 128-column ones, with the columns past D
+ *   read as zeros (extra tensor-core work, exact results).
  * scale. Finite and > 0 (1/sqrt(D) in the usual use); else FA_ERR_INVALID_ARG.
  * Sizes. B, H, Sq, Sk >= 1; B*H*Sq and B*H*Sk below 2^31.
  * Alignment. Every tensor base address 16-byte aligned and every stride a
@@ -172,10 +176,10 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
                    int causal, int dtype, fa_stream_t stream);
 
 /* Bytes of device workspace fa_bwd needs: an fp32 dq accumulator
-   [B, H, Sq_pad, D], the fp32 row terms Dvec_i = sum_d dO_id O_id
+   [B, H, Sq_pad, Dk], the fp32 row terms Dvec_i = sum_d dO_id O_id
    [B, H, Sq_pad] and the fp32 logsumexp in base 2 [B, H, Sq_pad], where
-   Sq_pad is Sq rounded up to a multiple of 128. Returns 0 for sizes < 1 or on
-   overflow. */
+   Sq_pad is Sq rounded up to a multiple of 128 and Dk is the kernel width
+   (64 for D <= 64, else 128). Returns 0 for sizes < 1 or on overflow. */
 size_t fa_bwd_workspace_size(int B, int H, int Sq, int D);
 
 /* Synchronises the current device, returns the status word recorded by

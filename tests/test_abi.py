@@ -37,6 +37,9 @@ def test_workspace_size(fa_lib):
     # dq accumulator (fp32, rows padded to 128) + Dvec + base-2 LSE (fp32)
     assert fa.fa_bwd_workspace_size(1, 2, 128, 64) == 2 * 128 * 64 * 4 + 2 * 2 * 128 * 4
     assert fa.fa_bwd_workspace_size(2, 12, 2000, 64) == 24 * 2048 * 64 * 4 + 2 * 24 * 2048 * 4
+    # head_dim below 64 uses the 64-wide accumulator, above 64 the 128-wide one
+    assert fa.fa_bwd_workspace_size(1, 1, 128, 32) == fa.fa_bwd_workspace_size(1, 1, 128, 64)
+    assert fa.fa_bwd_workspace_size(1, 1, 128, 96) == 128 * (128 + 2) * 4
     assert fa.fa_bwd_workspace_size(0, 1, 1, 64) == 0
     assert fa.fa_bwd_workspace_size(1, 1, -5, 64) == 0
 
@@ -63,7 +66,8 @@ def bwd(**kw):
     (dict(B=0), -1), (dict(H=-1), -1), (dict(Sq=0), -1), (dict(Sk=0), -1),
     (dict(scale=0.0), -1), (dict(scale=-1.0), -1), (dict(scale=float("nan")), -1), (dict(scale=float("inf")), -1),
     (dict(causal=2), -1),
-    (dict(D=32), -2), (dict(D=96), -2), (dict(D=256), -2), (dict(dtype=2), -2), (dict(dtype=-1), -2),
+    (dict(D=4), -2), (dict(D=100), -2), (dict(D=136), -2), (dict(D=256), -2), (dict(D=0), -2),
+    (dict(dtype=2), -2), (dict(dtype=-1), -2),
     (dict(q=A + 8), -3), (dict(v=A + 2), -3), (dict(o=A + 4), -3), (dict(lse=A + 2), -3),
     (dict(B=1 << 16, H=1 << 16, Sq=1 << 10), -1),
 ])
@@ -73,7 +77,7 @@ def test_fwd_rejects(fa_lib, kw, code):
 
 @pytest.mark.parametrize("kw,code", [
     (dict(dO=None), -1), (dict(dq=None), -1), (dict(dk=None), -1), (dict(dv=None), -1), (dict(lse=None), -1),
-    (dict(D=80), -2), (dict(dtype=3), -2), (dict(dk=A + 8), -3), (dict(dO=A + 4), -3),
+    (dict(D=81), -2), (dict(D=144), -2), (dict(dtype=3), -2), (dict(dk=A + 8), -3), (dict(dO=A + 4), -3),
     (dict(ws=None), -7), (dict(ws_bytes=100), -7), (dict(ws=A + 16), -3),
 ])
 def test_bwd_rejects(fa_lib, kw, code):

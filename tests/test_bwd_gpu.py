@@ -27,6 +27,12 @@ def test_bwd_rectangular(D, causal, Sq, Sk):
                what=f"Sq{Sq} Sk{Sk} D{D} c{causal}")
 
 
+@pytest.mark.parametrize("D", [8, 32, 40, 72, 96, 120])
+@pytest.mark.parametrize("causal", [False, True])
+def test_bwd_other_head_dims(D, causal):
+    full_check(random_case(2, 2, 300, 257, D, torch.float16, 190 + D), causal, what=f"D{D} c{causal}")
+
+
 @pytest.mark.parametrize("scale", [0.02, 0.5])
 def test_bwd_scale(scale):
     full_check(random_case(1, 2, 300, 300, 128, torch.float16, 9), True, scale=scale, what=f"scale {scale}")

@@ -35,6 +35,13 @@ def test_fwd_rectangular(D, causal, Sq, Sk):
     _fwd_case(2, 3, Sq, Sk, D, torch.bfloat16, causal, seed=7 + Sq + Sk)
 
 
+@pytest.mark.parametrize("D", [8, 32, 40, 72, 96, 120])
+@pytest.mark.parametrize("causal", [False, True])
+def test_fwd_other_head_dims(D, causal):
+    # head_dim below the kernel width: the extra columns are read as zeros
+    _fwd_case(2, 2, 300, 257, D, torch.bfloat16, causal, seed=90 + D, scale=D ** -0.5)
+
+
 @pytest.mark.parametrize("scale", [0.01, 0.5, 1.0])
 def test_fwd_scale(scale):
     _fwd_case(1, 2, 300, 300, 64, torch.float16, True, seed=5, scale=scale)

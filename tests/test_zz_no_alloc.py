@@ -71,4 +71,4 @@ def test_noalloc_rejects_problems_beyond_its_scratch(fa_lib):
     assert "64 MiB" in fa.fa_strerror(st)
     # the ordinary argument checks still come first
     assert fa.fa_bwd_noalloc(None, A, A, A, A, A, A, A, A, 1, 1, 8, 8, 64, 0.1, 0, fa.FA_FP16, 0) == -1
-    assert fa.fa_bwd_noalloc(A, A, A, A, A, A, A, A, A, 1, 1, 8, 8, 96, 0.1, 0, fa.FA_FP16, 0) == -2
+    assert fa.fa_bwd_noalloc(A, A, A, A, A, A, A, A, A, 1, 1, 8, 8, 100, 0.1, 0, fa.FA_FP16, 0) == -2
