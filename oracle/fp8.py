@@ -78,3 +78,22 @@ def e4m3_p_rounding_bound(q, k, v, scale: float, causal: bool, b: int, h: int, r
     h_err = np.where(allowed, np.maximum(2.0 ** -4 * p, 2.0 ** -10), 0.0)
     return (h_err @ np.abs(_f64(v[b, :, h]))) / l
 
+
+
+def e4m3_p_rounding_variance(q, k, v, scale: float, causal: bool, b: int, h: int, rows):
+    """Upper bound on the expected squared change of O[b, rows, h, :] from the
+    same rounding, modelling each rounding error as uniform on [-u, u] (variance
+    u^2 / 3) and independent across keys, with u the bound on the error used by
+    ``e4m3_p_rounding_bound``:
+        sum_j max(2^-4 P_ij, 2^-10)^2 v_jd^2 / (3 l_i^2).
+    Returns [len(rows), D].
+    """
+    x = _rows_scores(q, k, scale, causal, b, h, rows)
+    mx = np.max(x, axis=-1, keepdims=True)
+    mx = np.where(np.isfinite(mx), mx, 0.0)
+    p = np.exp(x - mx)
+    allowed = np.isfinite(x)
+    l = np.sum(p, axis=-1, keepdims=True)
+    l = np.where(l > 0, l, 1.0)
+    u = np.where(allowed, np.maximum(2.0 ** -4 * p, 2.0 ** -10), 0.0)
+    return ((u * u) @ (_f64(v[b, :, h]) ** 2)) / (3.0 * l * l)

@@ -150,7 +150,33 @@ def check_p_rounding_bound(f8, seed=22):
         assert math.isclose(err, want_frac * bound, rel_tol=1e-9), (p2, err, bound)
 
 
+def check_p_rounding_variance(f8, seed=23):
+    """Brute-force rounding of P' = c P, with c = 2^u drawn per row, over many
+    rows: the mean squared change of O stays below the variance bound and above
+    a quarter of it (for normal values the half-unit error is between 2^-5 P
+    and 2^-4 P, so the bound overstates the variance by a factor 1 to 4)."""
+    bts = np.arange(127)
+    vals = _torch_decode(bts)
+    rng = np.random.default_rng(seed)
+    Sq, Sk, D = 64, 96, 4
+    q = rng.standard_normal((1, Sq, 1, D)) * 1.5
+    k = rng.standard_normal((1, Sk, 1, D)) * 1.5
+    v = rng.standard_normal((1, Sk, 1, D)) * 3.0
+    scale = 0.8
+    rows = np.arange(Sq)
+    var = f8.e4m3_p_rounding_variance(q, k, v, scale, False, 0, 0, rows)
+    x = scale * (q[0, :, 0] @ k[0, :, 0].T)
+    p = np.exp(x - x.max(-1, keepdims=True))
+    l = p.sum(-1, keepdims=True)
+    o = (p @ v[0, :, 0]) / l
+    c = 2.0 ** rng.uniform(0, 8, size=(Sq, 1))
+    pr = _round_e4m3_bruteforce(c * p, vals, bts) / c
+    err2 = (((pr @ v[0, :, 0]) / l - o) ** 2).sum()
+    ratio = err2 / var.sum()
+    assert 0.25 <= ratio <= 1.0, ratio
+
+
 ALL_FP8_CHECKS = [
     check_e4m3_closed_forms, check_e4m3_all_bytes_vs_torch, check_e4m3_order_and_sign,
-    check_attention_vs_sdpa, check_descale_algebra, check_p_rounding_bound,
+    check_attention_vs_sdpa, check_descale_algebra, check_p_rounding_bound, check_p_rounding_variance,
 ]

@@ -24,9 +24,16 @@ MUTANTS = {
     "no_sign": ("return np.where(s == 1, -mag, mag)", "return mag"),
     "descale_ignored": ("return decode_e4m3(b) * float(descale)", "return decode_e4m3(b)"),
     "v_takes_k_descale": ("dequantize(v8, v_descale), scale, causal)", "dequantize(v8, k_descale), scale, causal)"),
-    "bound_half_ulp_2m5": ("np.maximum(2.0 ** -4 * p, 2.0 ** -10)", "np.maximum(2.0 ** -5 * p, 2.0 ** -10)"),
-    "bound_no_subnormal": ("np.maximum(2.0 ** -4 * p, 2.0 ** -10)", "2.0 ** -4 * p"),
+    "bound_half_ulp_2m5": ("h_err = np.where(allowed, np.maximum(2.0 ** -4 * p, 2.0 ** -10), 0.0)",
+                           "h_err = np.where(allowed, np.maximum(2.0 ** -5 * p, 2.0 ** -10), 0.0)"),
+    "bound_no_subnormal": ("h_err = np.where(allowed, np.maximum(2.0 ** -4 * p, 2.0 ** -10), 0.0)",
+                           "h_err = np.where(allowed, 2.0 ** -4 * p, 0.0)"),
+    "variance_half_ulp_2m5": ("u = np.where(allowed, np.maximum(2.0 ** -4 * p, 2.0 ** -10), 0.0)",
+                              "u = np.where(allowed, np.maximum(2.0 ** -5 * p, 2.0 ** -10), 0.0)"),
     "bound_signed_v": ("(h_err @ np.abs(_f64(v[b, :, h]))) / l", "(h_err @ _f64(v[b, :, h])) / l"),
+    "variance_no_third": ("/ (3.0 * l * l)", "/ (l * l)"),
+    "variance_not_squared": ("((u * u) @ (_f64(v[b, :, h]) ** 2))", "((u * u) @ np.abs(_f64(v[b, :, h])))"),
+    "variance_one_l": ("/ (3.0 * l * l)", "/ (3.0 * l)"),
     "bound_no_l": ("(h_err @ np.abs(_f64(v[b, :, h]))) / l", "(h_err @ np.abs(_f64(v[b, :, h])))"),
 }
 
