@@ -63,22 +63,27 @@ fa_tensor dense(const void* p, int S, int H, int D) {
   return t;
 }
 
-// 4-D tiled map over a [B, S, H, D] view: dims (D, S, H, B), box (64, rows, 1, 1),
-// 128-byte swizzle, out-of-range rows read as zeros.
+// 4-D tiled map over a [B, S, H, D] view: dims (D, S, H, B), box (128 bytes of
+// columns, rows, 1, 1), 128-byte swizzle, out-of-range rows and columns read
+// as zeros. `dtype` is FA_FP16, FA_BF16 or kE4M3 (one byte per element).
+constexpr int kE4M3 = 100;
 int make_map(CUtensorMap* map, const fa_tensor& t, int B, int S, int H, int D, int dtype, int box_rows) {
   auto fn = encode_fn();
   if (!fn) return FA_ERR_CUDA;
+  const int esz = dtype == kE4M3 ? 1 : 2;
+  const CUtensorMapDataType dt = dtype == kE4M3   ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                 : dtype == FA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                    : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   cuuint64_t dims[4] = {cuuint64_t(D), cuuint64_t(S), cuuint64_t(H), cuuint64_t(B)};
-  cuuint64_t strides[3] = {cuuint64_t(t.stride_s) * 2, cuuint64_t(t.stride_h) * 2, cuuint64_t(t.stride_b) * 2};
+  cuuint64_t strides[3] = {cuuint64_t(t.stride_s) * esz, cuuint64_t(t.stride_h) * esz, cuuint64_t(t.stride_b) * esz};
   // A stride the driver rejects (0 for an extent-1 axis) is replaced by a
   // harmless positive one: with extent 1 it is never stepped over.
   if (S == 1 && strides[0] == 0) strides[0] = 16;
   if (H == 1 && strides[1] == 0) strides[1] = 16;
   if (B == 1 && strides[2] == 0) strides[2] = 16;
-  cuuint32_t box[4] = {64, cuuint32_t(box_rows), 1, 1};
+  cuuint32_t box[4] = {cuuint32_t(128 / esz), cuuint32_t(box_rows), 1, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = fn(map, dtype == FA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4,
-                  t.ptr, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  CUresult r = fn(map, dt, 4, t.ptr, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
@@ -119,6 +124,40 @@ int launch_fwd(const fa_fwd_params* p, cudaStream_t stream) {
   a.Sq = p->Sq;
   a.Sk = p->Sk;
   a.scale_log2 = p->scale * 1.4426950408889634f;
+  a.o_scale = 1.f;
+  a.causal = p->causal;
+  a.n_qblocks = (p->Sq + 255) / 256;
+  a.d = p->D;
+  const unsigned grid = unsigned(int64_t(a.n_qblocks) * p->B * p->H);
+  kern<<<grid, L::kThreads, L::SMEM_ALLOC, stream>>>(mq, mk, mv, a);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+// e4m3 inputs: one kernel width (128 bytes = 128 columns) for every head_dim.
+template <bool OUT_BF16>
+int launch_fwd_fp8(const fa_fwd_fp8_params* p, cudaStream_t stream) {
+  using L = fa::FwdLayout<128, 1>;
+  static bool done[kMaxDevices] = {};
+  auto* kern = &fa::fa_fwd_kernel<128, OUT_BF16, true>;
+  int st = prepare(kern, L::SMEM_ALLOC, done);
+  if (st != FA_OK) return st;
+  CUtensorMap mq, mk, mv;
+  if ((st = make_map(&mq, p->q, p->B, p->Sq, p->H, p->D, kE4M3, 128)) != FA_OK) return st;
+  if ((st = make_map(&mk, p->k, p->B, p->Sk, p->H, p->D, kE4M3, 128)) != FA_OK) return st;
+  if ((st = make_map(&mv, p->v, p->B, p->Sk, p->H, p->D, kE4M3, 128)) != FA_OK) return st;
+  fa::FwdArgs a;
+  a.o = p->o.ptr;
+  a.lse = p->lse;
+  a.o_sb = p->o.stride_b;
+  a.o_ss = p->o.stride_s;
+  a.o_sh = p->o.stride_h;
+  a.B = p->B;
+  a.H = p->H;
+  a.Sq = p->Sq;
+  a.Sk = p->Sk;
+  // S = (q8 . k8) * q_descale * k_descale; O = (P v8 / l) * v_descale.
+  a.scale_log2 = float(double(p->scale) * p->q_descale * p->k_descale * 1.4426950408889634);
+  a.o_scale = p->v_descale;
   a.causal = p->causal;
   a.n_qblocks = (p->Sq + 255) / 256;
   a.d = p->D;
@@ -217,7 +256,7 @@ const char* fa_strerror(int s) {
   switch (s) {
     case FA_OK: return "ok";
     case FA_ERR_INVALID_ARG: return "invalid argument (null pointer, size < 1, scale or causal flag)";
-    case FA_ERR_UNSUPPORTED: return "unsupported dtype or head_dim (fp16/bf16; D a multiple of 8 in [8, 128])";
+    case FA_ERR_UNSUPPORTED: return "unsupported dtype or head_dim (fp16/bf16: D a multiple of 8 in [8, 128]; e4m3: a multiple of 16)";
     case FA_ERR_MISALIGNED: return "tensor base or stride not 16-byte aligned";
     case FA_ERR_CUDA: return "CUDA runtime or driver call failed";
     case FA_ERR_TIMEOUT: return "device-side pipeline wait exceeded its time limit";
@@ -262,6 +301,52 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
   p.causal = causal;
   p.dtype = dtype;
   return fa_fwd_ex(&p, stream);
+}
+
+int fa_fwd_fp8_ex(const fa_fwd_fp8_params* p, fa_stream_t stream) {
+  if (p == nullptr) return FA_ERR_INVALID_ARG;
+  if (p->o_dtype != FA_FP16 && p->o_dtype != FA_BF16) return FA_ERR_UNSUPPORTED;
+  int st = check_common(p->B, p->H, p->Sq, p->Sk, p->D, p->scale, p->causal, p->o_dtype);
+  if (st != FA_OK) return st;
+  if (p->D % 16) return FA_ERR_UNSUPPORTED;
+  for (float f : {p->q_descale, p->k_descale, p->v_descale})
+    if (!(std::isfinite(f) && f > 0.f)) return FA_ERR_INVALID_ARG;
+  if (!std::isfinite(float(double(p->scale) * p->q_descale * p->k_descale * 1.4426950408889634)))
+    return FA_ERR_INVALID_ARG;
+  const fa_tensor* in[3] = {&p->q, &p->k, &p->v};
+  for (const fa_tensor* v : in) {
+    if ((st = check_view(*v)) != FA_OK) return st;
+    if ((v->stride_b % 16) || (v->stride_s % 16) || (v->stride_h % 16)) return FA_ERR_MISALIGNED;
+  }
+  if ((st = check_view(p->o)) != FA_OK) return st;
+  if (p->lse == nullptr) return FA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(p->lse) & 3u) return FA_ERR_MISALIGNED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return p->o_dtype == FA_BF16 ? launch_fwd_fp8<true>(p, s) : launch_fwd_fp8<false>(p, s);
+}
+
+int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Sq, int Sk, int D,
+               float scale, float q_descale, float k_descale, float v_descale, int causal, int o_dtype,
+               fa_stream_t stream) {
+  fa_fwd_fp8_params p;
+  std::memset(&p, 0, sizeof(p));
+  p.q = dense(q, Sq, H, D);
+  p.k = dense(k, Sk, H, D);
+  p.v = dense(v, Sk, H, D);
+  p.o = dense(o, Sq, H, D);
+  p.lse = lse;
+  p.B = B;
+  p.H = H;
+  p.Sq = Sq;
+  p.Sk = Sk;
+  p.D = D;
+  p.scale = scale;
+  p.q_descale = q_descale;
+  p.k_descale = k_descale;
+  p.v_descale = v_descale;
+  p.causal = causal;
+  p.o_dtype = o_dtype;
+  return fa_fwd_fp8_ex(&p, stream);
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int Sq, int D) {

@@ -64,7 +64,8 @@ struct FwdArgs {
   int64_t o_sb, o_ss, o_sh;  // element strides of o
   int B, H, Sq, Sk;
   int d;             // head_dim of the tensors (<= the kernel's padded D; columns past it read as 0)
-  float scale_log2;  // scale * log2(e)
+  float scale_log2;  // scale * log2(e) (times the Q and K descale factors for e4m3 inputs)
+  float o_scale;     // factor applied to O with 1/l: 1, or V's descale factor for e4m3 inputs
   int causal;
   int n_qblocks;     // ceil(Sq / 256)
 };

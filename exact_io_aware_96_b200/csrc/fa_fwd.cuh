@@ -38,13 +38,15 @@
 
 namespace fa {
 
-template <int D>
+// ESZ: bytes per Q/K/V element (2 for fp16/bf16, 1 for e4m3).
+template <int D, int ESZ = 2>
 struct FwdLayout {
   static constexpr int kThreads = 320;
-  static constexpr int KB = D / 64;           // 128-byte column blocks per row
-  static constexpr int TILE = 128 * D * 2;    // bytes of one 128-row tile
-  static constexpr int BLK = 128 * 128;       // bytes of one 128-row x 64-column block
-  static constexpr int STAGES = (D == 128) ? 2 : 4;
+  static constexpr int RB = D * ESZ;          // bytes of one tile row
+  static constexpr int KB = RB / 128;         // 128-byte column blocks per row
+  static constexpr int TILE = 128 * RB;       // bytes of one 128-row tile
+  static constexpr int BLK = 128 * 128;       // bytes of one 128-row x 128-byte block
+  static constexpr int STAGES = (RB == 256) ? 2 : 4;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + 2 * TILE;
   static constexpr int OFF_V = OFF_K + STAGES * TILE;
@@ -66,11 +68,17 @@ __device__ __forceinline__ int fwd_kv_blocks(int r0, int Sq, int Sk, int causal)
   return min(nk, last / 128 + 1);
 }
 
-template <int D, bool BF16>
+// FP8 = false: Q, K, V and O are fp16 (BF16 = false) or bf16 (BF16 = true).
+// FP8 = true: Q, K, V are e4m3 with per-tensor descale factors (folded into
+// a.scale_log2 and a.o_scale), P is rounded to e4m3 for the P V product, and O
+// is bf16 or fp16 as BF16 says.
+template <int D, bool BF16, bool FP8 = false>
 __global__ void __launch_bounds__(320, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdArgs a) {
-  using L = FwdLayout<D>;
+  static_assert(!FP8 || D == 128, "e4m3 tiles are one 128-byte swizzle block wide");
+  using L = FwdLayout<D, FP8 ? 1 : 2>;
+  constexpr int KCOL = 128 / (FP8 ? 1 : 2);  // elements per 128-byte column block
   using namespace sm100;
   constexpr int S = L::STAGES;
 
@@ -145,7 +153,7 @@ __global__ void __launch_bounds__(320, 1)
       for (int t = 0; t < 2; ++t)
         if (nkv[t] > 0)
           for (int kb = 0; kb < L::KB; ++kb)
-            tma_load_4d(smem + L::OFF_Q + t * L::TILE + kb * L::BLK, &tmQ, q_full, kb * 64, q0 + 128 * t, h, b);
+            tma_load_4d(smem + L::OFF_Q + t * L::TILE + kb * L::BLK, &tmQ, q_full, kb * KCOL, q0 + 128 * t, h, b);
       int j = 0;
       for (; j < nmax; ++j) {
         const int st = j % S;
@@ -153,14 +161,14 @@ __global__ void __launch_bounds__(320, 1)
         if (!wait_bar(&k_empty[st], ph ^ 1, abort_flag, kRoleLoader, j)) break;
         mbar_arrive_expect_tx(&k_full[st], L::TILE);
         for (int kb = 0; kb < L::KB; ++kb)
-          tma_load_4d(smem + L::OFF_K + st * L::TILE + kb * L::BLK, &tmK, &k_full[st], kb * 64, j * 128, h, b);
+          tma_load_4d(smem + L::OFF_K + st * L::TILE + kb * L::BLK, &tmK, &k_full[st], kb * KCOL, j * 128, h, b);
         if (!wait_bar(&v_empty[st], ph ^ 1, abort_flag, kRoleLoader, j)) {
           ++j;  // K_j was issued
           break;
         }
         mbar_arrive_expect_tx(&v_full[st], L::TILE);
         for (int kb = 0; kb < L::KB; ++kb)
-          tma_load_4d(smem + L::OFF_V + st * L::TILE + kb * L::BLK, &tmV, &v_full[st], kb * 64, j * 128, h, b);
+          tma_load_4d(smem + L::OFF_V + st * L::TILE + kb * L::BLK, &tmV, &v_full[st], kb * KCOL, j * 128, h, b);
       }
       if (*abort_flag) {
         // Let the copies already issued land before the CTA exits.
@@ -174,8 +182,8 @@ __global__ void __launch_bounds__(320, 1)
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && nmax > 0) {
-      const uint32_t idS = idesc_f16(BF16, 128, 128, 0, 0);
-      const uint32_t idO = idesc_f16(BF16, 128, D, 0, 1);
+      const uint32_t idS = FP8 ? idesc_e4m3(128, 128, 0, 0) : idesc_f16(BF16, 128, 128, 0, 0);
+      const uint32_t idO = FP8 ? idesc_e4m3(128, D, 0, 1) : idesc_f16(BF16, 128, D, 0, 1);
       const uint32_t sQ = smem_u32(smem + L::OFF_Q);
       const uint32_t sK = smem_u32(smem + L::OFF_K);
       const uint32_t sV = smem_u32(smem + L::OFF_V);
@@ -183,17 +191,27 @@ __global__ void __launch_bounds__(320, 1)
         const uint32_t qa = sQ + t * L::TILE;
         const uint32_t ka = sK + st * L::TILE;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
+        for (int kk = 0; kk < L::RB / 32; ++kk) {  // 32 bytes of K per instruction
           const uint32_t o = (kk >> 2) * L::BLK + (kk & 3) * 32;
-          mma_ss(tmem + t * 128, desc_sw128(qa + o, 16, 1024), desc_sw128(ka + o, 16, 1024), idS, kk > 0);
+          if constexpr (FP8)
+            mma_ss_f8(tmem + t * 128, desc_sw128(qa + o, 16, 1024), desc_sw128(ka + o, 16, 1024), idS, kk > 0);
+          else
+            mma_ss(tmem + t * 128, desc_sw128(qa + o, 16, 1024), desc_sw128(ka + o, 16, 1024), idS, kk > 0);
         }
       };
       auto issue_PV = [&](int t, int st, int acc) {
         const uint32_t va = sV + st * L::TILE;
+        // P occupies 8 TMEM columns per instruction (16 keys of 16-bit, 32
+        // keys of e4m3); V advances by as many 128-byte rows.
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + 256 + t * D, tmem + t * 128 + kk * 8, desc_sw128(va + kk * 2048, L::BLK, 1024), idO,
-                 (acc || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < (FP8 ? 4 : 8); ++kk) {
+          if constexpr (FP8)
+            mma_ts_f8(tmem + 256 + t * D, tmem + t * 128 + kk * 8, desc_sw128(va + kk * 4096, L::BLK, 1024), idO,
+                      (acc || kk > 0) ? 1u : 0u);
+          else
+            mma_ts(tmem + 256 + t * D, tmem + t * 128 + kk * 8, desc_sw128(va + kk * 2048, L::BLK, 1024), idO,
+                   (acc || kk > 0) ? 1u : 0u);
+        }
       };
       bool ok = wait_bar(q_full, 0, abort_flag, kRoleMma, -1) && wait_bar(&k_full[0], 0, abort_flag, kRoleMma, 0);
       if (ok) {
@@ -315,8 +333,9 @@ __global__ void __launch_bounds__(320, 1)
       const uint64_t negmu2 = f2(-mu, -mu);
       uint64_t acc0 = f2(0.f, 0.f), acc1 = f2(0.f, 0.f);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {  // 32 columns at a time -> 16 packed P words
+      for (int q = 0; q < 4; ++q) {  // 32 columns at a time -> 16 (8 for e4m3) packed P words
         uint32_t pw[16];
+        float h0 = 0.f, h1 = 0.f;  // e4m3: the even pair, packed with the odd one
 #pragma unroll
         for (int cc = 0; cc < 16; ++cc) {
           const int c = 16 * q + cc;
@@ -335,9 +354,20 @@ __global__ void __launch_bounds__(320, 1)
             acc0 = add2(acc0, e);
           float e0, e1;
           f2_split(e, e0, e1);
-          pw[cc] = pack2<BF16>(e0, e1);
+          if constexpr (FP8) {
+            if (cc & 1)
+              pw[cc >> 1] = pack4_e4m3(h0, h1, e0, e1);
+            else
+              h0 = e0, h1 = e1;
+          } else {
+            pw[cc] = pack2<BF16>(e0, e1);
+          }
         }
-        tmem_st16(tS + 16 * q, pw);  // S columns [0, 64) were read already
+        // Every S column of this row was read into x[] already.
+        if constexpr (FP8)
+          tmem_st8(tS + 8 * q, *reinterpret_cast<const uint32_t(*)[8]>(pw));
+        else
+          tmem_st16(tS + 16 * q, pw);
       }
       {
         const uint64_t acc = add2(acc0, acc1);
@@ -354,7 +384,7 @@ __global__ void __launch_bounds__(320, 1)
     if (ok && !*abort_flag && r0 < a.Sq) {
       const bool valid = row < a.Sq;
       const bool has = (m != -INFINITY) && l > 0.f;  // m stays -inf only for rows with no allowed key
-      const float inv_l = has ? 1.f / l : 0.f;
+      const float inv_l = has ? a.o_scale / l : 0.f;  // o_scale: V's descale (1 for 16-bit inputs)
       uint16_t* orow = reinterpret_cast<uint16_t*>(a.o) + static_cast<int64_t>(b) * a.o_sb +
                        static_cast<int64_t>(row) * a.o_ss + static_cast<int64_t>(h) * a.o_sh;
       if (n > 0) {

@@ -23,8 +23,8 @@ STATUS = {
     -8: "FA_ERR_SCRATCH_LIMIT",
 }
 FA_NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
-EXPORTED = ("fa_fwd", "fa_fwd_ex", "fa_bwd", "fa_bwd_ex", "fa_bwd_noalloc", "fa_bwd_workspace_size",
-            "fa_last_device_status", "fa_strerror", "fa_version")
+EXPORTED = ("fa_fwd", "fa_fwd_ex", "fa_fwd_fp8", "fa_fwd_fp8_ex", "fa_bwd", "fa_bwd_ex", "fa_bwd_noalloc",
+            "fa_bwd_workspace_size", "fa_last_device_status", "fa_strerror", "fa_version")
 
 
 class FaTensor(ctypes.Structure):
@@ -38,6 +38,15 @@ class FwdParams(ctypes.Structure):
                 ("B", ctypes.c_int), ("H", ctypes.c_int), ("Sq", ctypes.c_int), ("Sk", ctypes.c_int),
                 ("D", ctypes.c_int), ("scale", ctypes.c_float), ("causal", ctypes.c_int),
                 ("dtype", ctypes.c_int)]
+
+
+class FwdFp8Params(ctypes.Structure):
+    _fields_ = [("q", FaTensor), ("k", FaTensor), ("v", FaTensor), ("o", FaTensor),
+                ("lse", ctypes.c_void_p),
+                ("B", ctypes.c_int), ("H", ctypes.c_int), ("Sq", ctypes.c_int), ("Sk", ctypes.c_int),
+                ("D", ctypes.c_int), ("scale", ctypes.c_float),
+                ("q_descale", ctypes.c_float), ("k_descale", ctypes.c_float), ("v_descale", ctypes.c_float),
+                ("causal", ctypes.c_int), ("o_dtype", ctypes.c_int)]
 
 
 class BwdParams(ctypes.Structure):
@@ -71,6 +80,10 @@ def lib():
         L.fa_fwd.restype = i
         L.fa_fwd_ex.argtypes = [ctypes.POINTER(FwdParams), vp]
         L.fa_fwd_ex.restype = i
+        L.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, f, f, f, i, i, vp]
+        L.fa_fwd_fp8.restype = i
+        L.fa_fwd_fp8_ex.argtypes = [ctypes.POINTER(FwdFp8Params), vp]
+        L.fa_fwd_fp8_ex.restype = i
         L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp, sz, vp]
         L.fa_bwd.restype = i
         L.fa_bwd_ex.argtypes = [ctypes.POINTER(BwdParams), vp]
@@ -96,6 +109,16 @@ def fa_fwd(q, k, v, o, lse, B, H, Sq, Sk, D, scale, causal, dtype, stream=0) -> 
 
 def fa_fwd_ex(params: FwdParams, stream=0) -> int:
     return lib().fa_fwd_ex(ctypes.byref(params), stream)
+
+
+def fa_fwd_fp8(q, k, v, o, lse, B, H, Sq, Sk, D, scale, q_descale, k_descale, v_descale, causal, o_dtype,
+               stream=0) -> int:
+    return lib().fa_fwd_fp8(q, k, v, o, lse, B, H, Sq, Sk, D, scale, q_descale, k_descale, v_descale, causal,
+                            o_dtype, stream)
+
+
+def fa_fwd_fp8_ex(params: FwdFp8Params, stream=0) -> int:
+    return lib().fa_fwd_fp8_ex(ctypes.byref(params), stream)
 
 
 def fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, Sq, Sk, D, scale, causal, dtype,
@@ -177,6 +200,36 @@ def forward(q, k, v, causal=False, scale=None, out=None, lse=None, stream=None):
     st = fa_fwd_ex(p, _stream(stream))
     if st != FA_OK:
         raise FaError(st, "fa_fwd_ex")
+    return out, lse
+
+
+def forward_fp8(q, k, v, q_descale, k_descale, v_descale, causal=False, scale=None,
+                out_dtype=torch.bfloat16, out=None, lse=None, stream=None):
+    """O, LSE from e4m3 tensors: the values attended over are q * q_descale,
+    k * k_descale, v * v_descale. q, k, v are torch.float8_e4m3fn (or uint8
+    holding E4M3 bytes) [B, S, H, D] CUDA views; O is ``out_dtype``."""
+    B, Sq, H, D = q.shape
+    Sk = k.shape[1]
+    for t in (q, k, v):
+        if t.dtype not in (torch.float8_e4m3fn, torch.uint8):
+            raise TypeError(f"e4m3 tensors (torch.float8_e4m3fn or uint8 bytes) only, got {t.dtype}")
+    od = _DT.get(out_dtype)
+    if od is None:
+        raise TypeError(f"out_dtype must be fp16 or bf16, got {out_dtype}")
+    if scale is None:
+        scale = D ** -0.5
+    if out is None:
+        out = torch.empty((B, Sq, H, D), dtype=out_dtype, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, H, Sq), dtype=torch.float32, device=q.device)
+    if lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous fp32 [B, H, Sq] tensor")
+    p = FwdFp8Params(_view(q), _view(k), _view(v), _view(out), lse.data_ptr(),
+                     B, H, Sq, Sk, D, float(scale), float(q_descale), float(k_descale), float(v_descale),
+                     int(bool(causal)), od)
+    st = fa_fwd_fp8_ex(p, _stream(stream))
+    if st != FA_OK:
+        raise FaError(st, "fa_fwd_fp8_ex")
     return out, lse
 
 

@@ -17,6 +17,9 @@ Workloads (shapes from the usage snippets of the pages, see the legend below):
 * ``c5``  B=1  H=16 S=16384 D=128 bf16 causal / non-causal  seed 4, Q and K
   drawn N(0, 2^2) to widen the softmax range
 
+The e4m3 forward takes a workload's fp32 draws (same recipe, dtype ignored)
+through ``quantize_e4m3``: one descale per tensor, max |x| mapped to 448.
+
 Draw recipe: ``torch.Generator('cpu').manual_seed(seed)``; ``torch.randn`` in
 fp32, in the order Q, K, V, dO (packed: qkv then dO); multiply Q and K by
 ``qk_std``; cast to the workload dtype. All tensors are [B, S, H, D].
@@ -113,6 +116,19 @@ def random_case(B, H, Sq, Sk, D, dtype, seed, qk_std=1.0):
     v = draw((B, Sk, H, D), g, dtype)
     do = draw((B, Sq, H, D), g, dtype)
     return {"q": q, "k": k, "v": v, "do": do}
+
+
+def quantize_e4m3(x: torch.Tensor):
+    """Per-tensor E4M3 encoding for the e4m3 forward's inputs: returns (bytes
+    as a torch.uint8 tensor, descale) with x ~= value(bytes) * descale, the
+    descale (an fp32 number) chosen so that max |x| lands on 448, the largest
+    finite E4M3 value. The rounding is torch's float8_e4m3fn cast. This
+    prepares inputs; it is not a step of the attention."""
+    xf = x.float()
+    amax = float(xf.abs().max()) if xf.numel() else 0.0
+    descale = float(torch.tensor(amax / 448.0 if amax > 0 else 1.0, dtype=torch.float32))
+    y = (xf / descale).clamp(-448.0, 448.0).to(torch.float8_e4m3fn)
+    return y.view(torch.uint8), descale
 
 
 def sample_rows(S: int, block: int, n_random: int, seed: int):

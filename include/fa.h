@@ -22,6 +22,9 @@
  *        matrix products in the backward), §4 (flash_attn_func on
  *        (batch, seq_len, num_heads, head_dim), causal flag), §5 (fp32 inputs
  *        are rejected).
+ *   [P5] the FlashAttention "IO感知" overview (0539edu.com/news/165270),
+ *        sections "H100的FP8加速能力" and "未来展望" (an FP8 data type in
+ *        FlashAttention-3): fa_fwd_fp8.
  *
  * Conventions shared by every entry point
  * ---------------------------------------
@@ -127,6 +130,50 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
 
 /* Forward on strided views (packed qkv and the like). Same semantics. */
 int fa_fwd_ex(const fa_fwd_params* p, fa_stream_t stream);
+
+/* e4m3 forward: the parameters of fa_fwd_fp8_ex. */
+typedef struct {
+  fa_tensor q, k, v; /* read, E4M3 bytes; strides in elements (= bytes) */
+  fa_tensor o;       /* written, o_dtype */
+  float* lse;        /* written, dense fp32 [B, H, Sq] */
+  int B, H, Sq, Sk, D;
+  float scale;
+  float q_descale, k_descale, v_descale; /* real value = stored E4M3 value * descale */
+  int causal;
+  int o_dtype; /* FA_FP16 or FA_BF16 */
+} fa_fwd_fp8_params;
+
+/* Forward from 8-bit floating-point inputs ([P5] sections "H100的FP8加速能力"
+   and "未来展望：FlashAttention-3带来的新可能": FlashAttention-3 adds an FP8
+   data type; the pages give no more than that, so the form below is this
+   library's reading).
+   q, k, v hold OCP E4M3 bytes (1 sign bit, 4 exponent bits with bias 7, 3
+   mantissa bits, largest finite value 448, no infinities) in the [B, S, H, D]
+   layout. The values attended over are q * q_descale, k * k_descale and
+   v * v_descale: one finite, positive factor per tensor. The result is the
+   same exact attention as fa_fwd on those values, computed as follows:
+   Q K^T is formed by the tensor cores with fp32 accumulation (products of two
+   E4M3 values are exact in fp32); the softmax runs in fp32 as in fa_fwd; the
+   probabilities P (relative to the running row maximum, at most 2^8) are
+   rounded to E4M3, round to nearest even, for the P V product; the row sum l
+   is taken over the unrounded P. So lse is as exact as fa_fwd's, and the
+   rounding of P moves each element of O by at most
+       sum_j max(2^-4 P_ij, 2^-10) |v_jd| / l_i
+   with P_ij = exp(scale q_i.k_j - max_j') relative to the row maximum and
+   l_i = sum_j P_ij. O is written as o_dtype, lse as in fa_fwd.
+   head_dim: D a multiple of 16 in [16, 128] (every tile is 128 bytes wide;
+   columns past D read as zeros). Alignment: base addresses 16-byte aligned,
+   strides of q, k and v multiples of 16 elements, of o multiples of 8.
+   Descale factors that are not finite and > 0 are FA_ERR_INVALID_ARG; an
+   o_dtype other than FA_FP16 or FA_BF16 is FA_ERR_UNSUPPORTED. Ownership,
+   asynchrony and error reporting as for fa_fwd. */
+int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
+               int B, int H, int Sq, int Sk, int D, float scale,
+               float q_descale, float k_descale, float v_descale, int causal,
+               int o_dtype, fa_stream_t stream);
+
+/* e4m3 forward on strided views. Same semantics. */
+int fa_fwd_fp8_ex(const fa_fwd_fp8_params* p, fa_stream_t stream);
 
 /* Backward ([P1] "性能引擎" recomputation; [P2] item 3; [P4] §3.1 logsumexp,
    §3.3 five matrix products). Given the forward's inputs, its outputs o and

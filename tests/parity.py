@@ -8,6 +8,7 @@ import numpy as np
 import torch
 
 import oracle
+import oracle.fp8
 from exact_io_aware_96_b200 import fa
 
 O_TOL = {torch.float16: 1e-2, torch.bfloat16: 2e-2}
@@ -83,3 +84,58 @@ def full_check(inp_cpu, causal, scale=None, backward=True, what=""):
     dq_r, dk_r, dv_r, _ = oracle.attention_backward(np64(q), np64(k), np64(v), np64(do), sc, causal)
     for name, g, r in (("dq", dq, dq_r), ("dk", dk, dk_r), ("dv", dv, dv_r)):
         check_grad(np64(g), r, f"{what} {name}")
+
+
+# ------------------------------------------------------------------ e4m3 forward
+# Half a unit in the last place of the output type, relative: bf16 keeps 8
+# significant bits, fp16 11.
+OUT_HALF_ULP = {torch.bfloat16: 2.0 ** -8, torch.float16: 2.0 ** -11}
+
+
+def run_fwd_fp8(q8, k8, v8, qd, kd, vd, causal, scale=None, out_dtype=torch.bfloat16):
+    o, lse = fa.forward_fp8(q8, k8, v8, qd, kd, vd, causal=causal, scale=scale, out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    st, detail = fa.fa_last_device_status()
+    assert st == 0, f"device status {st} {detail}"
+    return o, lse
+
+
+def check_fp8_o_lse(o_gpu, lse_gpu, qn, kn, vn, scale, causal, out_dtype, b, h, rows, what=""):
+    """O[b, rows, h] and LSE[b, h, rows] of the e4m3 forward against exact
+    attention on the dequantized inputs (qn, kn, vn fp64).
+
+    The kernel differs from exact attention by (1) rounding P to E4M3 before
+    the P V product, (2) the rounding of O to ``out_dtype``, (3) fp32
+    arithmetic and exp2 approximations (relative 2^-13 at most, below 2^-8 of
+    (1)). Two bars:
+    * every element within the worst case of (1) from
+      ``oracle.fp8.e4m3_p_rounding_bound`` (times 1 + 2^-8 for (3)), plus
+      (2), half an ulp of |O|;
+    * when at least 2048 elements are compared, the summed squared error
+      within twice the expected value of (1) + (2) (the oracle's variance bound
+      plus u^2 |O|^2 / 3), a bar that a wrong key, row or column breaks.
+    LSE does not see the rounding of P (the row sum uses the unrounded values):
+    the 16-bit path's bar applies.
+    """
+    o_gpu, lse_gpu = np.asarray(o_gpu, np.float64), np.asarray(lse_gpu, np.float64)
+    assert np.all(np.isfinite(o_gpu)), f"{what}: non-finite O"
+    o_ref, lse_ref = oracle.attention_forward_rows(qn, kn, vn, scale, causal, b, h, rows)
+    fin = np.isfinite(lse_ref)
+    assert np.array_equal(fin, np.isfinite(lse_gpu)), f"{what}: LSE finiteness differs"
+    assert np.all(lse_gpu[~fin] == -np.inf), f"{what}: masked rows must have LSE = -inf"
+    if fin.any():
+        lerr = np.max(np.abs(lse_gpu[fin] - lse_ref[fin]))
+        assert lerr <= LSE_TOL, f"{what}: LSE max-abs error {lerr:.3e} > {LSE_TOL}"
+    u = OUT_HALF_ULP[out_dtype]
+    bound = oracle.fp8.e4m3_p_rounding_bound(qn, kn, vn, scale, causal, b, h, rows)
+    tol = bound * (1 + 2.0 ** -8) + u * (np.abs(o_ref) + bound) + 1e-6
+    err = np.abs(o_gpu - o_ref)
+    bad = err > tol
+    assert not bad.any(), (f"{what}: {bad.sum()} elements beyond the e4m3 bound; worst err "
+                           f"{err[bad].max():.3e} vs tol {tol[bad][np.argmax(err[bad])]:.3e}")
+    if err.size >= 2048:
+        var = oracle.fp8.e4m3_p_rounding_variance(qn, kn, vn, scale, causal, b, h, rows)
+        expect = var.sum() + (u * u / 3.0) * np.sum(o_ref ** 2)
+        e2 = np.sum(err ** 2)
+        assert e2 <= 2.0 * expect + 1e-12, f"{what}: squared error {e2:.3e} > 2 x expected {expect:.3e}"
+    return float(err.max()) if err.size else 0.0

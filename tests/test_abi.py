@@ -84,6 +84,36 @@ def test_bwd_rejects(fa_lib, kw, code):
     assert bwd(**kw) == code
 
 
+def fwd_fp8(**kw):
+    args = dict(q=A, k=A, v=A, o=A, lse=A, B=1, H=2, Sq=128, Sk=128, D=64, scale=0.125,
+                qd=0.01, kd=0.02, vd=0.03, causal=0, o_dtype=fa.FA_BF16)
+    args.update(kw)
+    return fa.fa_fwd_fp8(*args.values())
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), -1), (dict(v=None), -1), (dict(lse=None), -1), (dict(Sk=0), -1), (dict(causal=-1), -1),
+    (dict(scale=0.0), -1), (dict(qd=0.0), -1), (dict(kd=-1.0), -1), (dict(vd=float("nan")), -1),
+    (dict(vd=float("inf")), -1), (dict(scale=1e30, qd=1e30), -1),
+    (dict(D=8), -2), (dict(D=72), -2), (dict(D=144), -2), (dict(o_dtype=2), -2), (dict(o_dtype=-1), -2),
+    (dict(q=A + 8), -3), (dict(o=A + 2), -3), (dict(lse=A + 1), -3),
+])
+def test_fwd_fp8_rejects(fa_lib, kw, code):
+    assert fwd_fp8(**kw) == code
+
+
+def test_fwd_fp8_strides(fa_lib):
+    t = fa.FaTensor(A, 3 * 512 * 12 * 64, 3 * 12 * 64, 64)
+    o = fa.FaTensor(A, 512 * 12 * 64, 12 * 64, 64)
+    p = fa.FwdFp8Params(t, t, t, o, A, 2, 12, 512, 512, 64, 0.125, 1.0, 1.0, 1.0, 0, fa.FA_BF16)
+    p.v = fa.FaTensor(A, 3 * 512 * 12 * 64, 3 * 12 * 64 + 8, 64)  # a multiple of 8 but not of 16 bytes
+    assert fa.fa_fwd_fp8_ex(p) == -3
+    p.v = t
+    p.o = fa.FaTensor(A, 512 * 12 * 64, 12 * 64 + 4, 64)
+    assert fa.fa_fwd_fp8_ex(p) == -3
+    assert fa_lib.fa_fwd_fp8_ex(None, None) == -1
+
+
 def test_strided_views_checked(fa_lib):
     t = fa.FaTensor(A, 3 * 512 * 12 * 64, 3 * 12 * 64, 64)
     p = fa.FwdParams(t, t, t, t, A, 2, 12, 512, 512, 64, 0.125, 0, fa.FA_FP16)

@@ -1,0 +1,120 @@
+"""e4m3 forward on the GPU: libfa.so's fa_fwd_fp8 (through the C ABI) against
+exact attention on the dequantized inputs (fp64 oracle), with the bars derived
+from the rounding of P to E4M3 (tests/parity.py, check_fp8_o_lse)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle.fp8
+from exact_io_aware_96_b200 import fa
+from exact_io_aware_96_b200.inputs import WORKLOADS, make_inputs, quantize_e4m3, random_case, sample_rows
+from tests.parity import check_fp8_o_lse, np64, run_fwd_fp8
+
+pytestmark = pytest.mark.gpu
+
+
+def _quantized(c):
+    out = {}
+    for n in ("q", "k", "v"):
+        b, d = quantize_e4m3(c[n])
+        out[n] = (b, d, oracle.fp8.dequantize(b.numpy(), d))
+    return out
+
+
+def _fp8_case(B, H, Sq, Sk, D, causal, seed, qk_std=1.0, scale=None, out_dtype=torch.bfloat16, what=""):
+    c = random_case(B, H, Sq, Sk, D, torch.float32, seed, qk_std)
+    z = _quantized(c)
+    sc = D ** -0.5 if scale is None else scale
+    o, lse = run_fwd_fp8(z["q"][0].cuda(), z["k"][0].cuda(), z["v"][0].cuda(), z["q"][1], z["k"][1], z["v"][1],
+                         causal, sc, out_dtype)
+    o, lse = np64(o), np64(lse)
+    rows = np.arange(Sq)
+    for b in range(B):
+        for h in range(H):
+            check_fp8_o_lse(o[b, :, h], lse[b, h], z["q"][2], z["k"][2], z["v"][2], sc, causal, out_dtype,
+                            b, h, rows, f"{what} B{B} H{H} Sq{Sq} Sk{Sk} D{D} c{causal} b{b} h{h}")
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("S", [1, 7, 63, 127, 128, 129, 256, 257, 640])
+def test_fp8_square(D, causal, S):
+    _fp8_case(1, 2, S, S, D, causal, seed=3000 + S)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("Sq,Sk", [(1, 300), (100, 37), (129, 700), (700, 129), (300, 1), (513, 255)])
+def test_fp8_rectangular(causal, Sq, Sk):
+    _fp8_case(2, 3, Sq, Sk, 128, causal, seed=50 + Sq + Sk)
+
+
+@pytest.mark.parametrize("D", [16, 32, 48, 80, 96, 112])
+def test_fp8_other_head_dims(D):
+    _fp8_case(2, 2, 300, 257, D, True, seed=400 + D)
+
+
+def test_fp8_fp16_output_and_scale():
+    _fp8_case(1, 2, 333, 333, 128, True, seed=8, out_dtype=torch.float16, what="fp16 out")
+    _fp8_case(1, 2, 333, 333, 64, False, seed=9, scale=0.05, what="scale 0.05")
+
+
+def test_fp8_wide_scores():
+    # Q, K ~ N(0, 2^2) and N(0, 4^2): peaked rows, the running max is raised often
+    _fp8_case(1, 2, 1000, 1000, 128, False, seed=21, qk_std=2.0)
+    _fp8_case(1, 2, 1000, 1000, 128, True, seed=22, qk_std=4.0)
+
+
+def test_fp8_descales_enter_as_stated():
+    """The same bytes with every descale doubled: scores x4 (so a different
+    softmax), O x2 relative to the real values; checked against the oracle."""
+    c = random_case(1, 2, 200, 200, 128, torch.float32, 31)
+    z = _quantized(c)
+    q8, k8, v8 = (z[n][0].cuda() for n in ("q", "k", "v"))
+    for f in (1.0, 2.0):
+        qd, kd, vd = (z[n][1] * f for n in ("q", "k", "v"))
+        o, lse = run_fwd_fp8(q8, k8, v8, qd, kd, vd, True, 128 ** -0.5)
+        qn, kn, vn = (oracle.fp8.dequantize(z[n][0].numpy(), d) for n, d in (("q", qd), ("k", kd), ("v", vd)))
+        o, lse = np64(o), np64(lse)
+        for h in range(2):
+            check_fp8_o_lse(o[0, :, h], lse[0, h], qn, kn, vn, 128 ** -0.5, True, torch.bfloat16, 0, h,
+                            np.arange(200), f"descale x{f} h{h}")
+
+
+def test_fp8_strided_packed_views():
+    """q, k, v as strided views into one [B, S, 3, H, D] byte tensor."""
+    B, S, H, D = 2, 300, 4, 64
+    c = random_case(B, H, S, S, D, torch.float32, 41)
+    z = _quantized(c)
+    packed = torch.stack([z["q"][0], z["k"][0], z["v"][0]], dim=2).cuda()
+    o, lse = run_fwd_fp8(packed[:, :, 0], packed[:, :, 1], packed[:, :, 2], z["q"][1], z["k"][1], z["v"][1],
+                         False, D ** -0.5)
+    o, lse = np64(o), np64(lse)
+    for b in range(B):
+        for h in range(H):
+            check_fp8_o_lse(o[b, :, h], lse[b, h], z["q"][2], z["k"][2], z["v"][2], D ** -0.5, False,
+                            torch.bfloat16, b, h, np.arange(S), f"packed b{b} h{h}")
+
+
+def test_fp8_repeatable():
+    c = random_case(1, 4, 777, 777, 128, torch.float32, 3)
+    z = _quantized(c)
+    args = [z[n][0].cuda() for n in ("q", "k", "v")] + [z[n][1] for n in ("q", "k", "v")]
+    o1, l1 = run_fwd_fp8(*args, True)
+    o2, l2 = run_fwd_fp8(*args, True)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_fp8_c4_full_size_sampled():
+    """c4's shape (B1 H8 S8192 D128, causal) from c4's draws, quantized per
+    tensor; O and LSE checked on sampled rows of every head."""
+    w = WORKLOADS["c4"]
+    g = torch.Generator("cpu").manual_seed(w.seed)
+    c = {n: torch.randn((w.B, w.S, w.H, w.D), generator=g, dtype=torch.float32) for n in ("q", "k", "v")}
+    z = _quantized(c)
+    o, lse = run_fwd_fp8(z["q"][0].cuda(), z["k"][0].cuda(), z["v"][0].cuda(), z["q"][1], z["k"][1], z["v"][1],
+                         True, w.scale)
+    o, lse = np64(o), np64(lse)
+    rows = np.array(sample_rows(w.S, 128, 118, w.seed))
+    for h in range(w.H):
+        check_fp8_o_lse(o[0, rows, h], lse[0, h, rows], z["q"][2], z["k"][2], z["v"][2], w.scale, True,
+                        torch.bfloat16, 0, h, rows, f"c4 e4m3 h{h}")
