@@ -9,6 +9,11 @@ for causal in the forward and 2.5x that in the backward (the backward's five
 matrix products against the forward's two).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--path fwd_bwd|fwd_e4m3]
+
+``--path fwd_e4m3`` times the e4m3 forward (fa_fwd_fp8) alone on c4's shape
+instead, with its own JSON line (peak: the measured bf16 figure times the
+nominal fp8/bf16 ratio of 2).
 
 N > 1 runs under torchrun, one process per GPU: every rank processes its own
 batch (weak scaling; attention heads are independent, so there is no
@@ -342,14 +347,168 @@ def run_ours(args, w, causal):
     return result if rank == 0 else None
 
 
+# ------------------------------------------------- our arm, e4m3 forward
+METRIC_E4M3 = "attention fwd TFLOP/s (e4m3 Q/K/V, bf16 O, causal, S=8K, d=128) and % of B200 dense fp8 peak"
+E4M3_PER_BF16 = 2.0  # nominal dense fp8 / bf16 tensor throughput (4.5 / 2.25 PFLOP/s)
+
+
+def run_ours_fwd_e4m3(args, w, causal):
+    """One step = one fa_fwd_fp8 call on the workload's shape, inputs encoded
+    per tensor to E4M3 (inputs.make_e4m3_inputs), O in bf16."""
+    import torch
+    import torch.distributed as dist
+    from exact_io_aware_96_b200 import fa
+    from exact_io_aware_96_b200.inputs import make_e4m3_inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    fa.lib()
+
+    lo, hi = rank_batch_slice(w.B * world, world, rank)
+    z = make_e4m3_inputs(w, B=hi - lo, seed=w.seed + rank)
+    q8, k8, v8 = (z[n][0].to(dev) for n in ("q", "k", "v"))
+    qd, kd, vd = (z[n][1] for n in ("q", "k", "v"))
+    B, S, H, D = q8.shape
+    o = torch.empty((B, S, H, D), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, H, S), dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        fa.forward_fp8(q8, k8, v8, qd, kd, vd, causal=causal, scale=w.scale, out=o, lse=lse, stream=stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    st, detail = fa.fa_last_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} {detail} after warm-up")
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    with ClockSampler(local) as clocks:
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        wall0 = time.perf_counter()
+        for i in range(args.steps):
+            flush.zero_()
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        wall = time.perf_counter() - wall0
+    st, detail = fa.fa_last_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} {detail} in the timed region")
+    t_dev = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev) / 1e3, dev)
+    ff = w.fwd_flops(causal) * (hi - lo) / w.B
+    value = ff * args.steps * world / t_dev / 1e12
+
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv = (t.cpu().pin_memory() for t in (q8, k8, v8))
+        ho, hl = torch.empty_like(o, device="cpu").pin_memory(), torch.empty_like(lse, device="cpu").pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
+        d2h = sum(t.numel() * t.element_size() for t in (ho, hl))
+
+        def e2e_step():
+            for src, dst in ((hq, q8), (hk, k8), (hv, v8)):
+                dst.copy_(src, non_blocking=True)
+            step()
+            for src, dst in ((o, ho), (lse, hl)):
+                dst.copy_(src, non_blocking=True)
+
+        for _ in range(max(1, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize()
+        n_e2e = max(3, min(args.steps, 50))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        e0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        t_e2e = max_over_ranks(e0.elapsed_time(e1) / 1e3, dev)
+        e2e = {"value": ff * n_e2e * world / t_e2e / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e}
+
+    peaks, peaks_src = load_peaks()
+    sustained = t_dev > 1.0
+    key = "bf16_tflops_sustained" if sustained else "bf16_tflops"
+    peak_tf = peaks[key] * E4M3_PER_BF16
+    achieved = ff / (t_dev / args.steps) / 1e12
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tpath):
+        with open(tpath) as f:
+            ent = json.load(f).get("fa_fwd_kernel_e4m3")
+        if ent and ent.get("source_hash") == kernel_source_hash("fa_fwd_kernel"):
+            traffic = ent.get("bytes_per_launch")
+    result = {
+        "metric": METRIC_E4M3, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": t_dev / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 (fp32 accumulate, bf16 out)", "data": "synthetic",
+        "config": {"workload": f"{w.name} shape, e4m3: B={w.B} H={w.H} S={w.S} D={w.D} causal={causal}, "
+                               "forward only (fa_fwd_fp8), per-tensor descales",
+                   "global_batch": w.B * world, "seq_len": w.S, "heads": w.H, "head_dim": w.D, "causal": causal,
+                   "parallelism": f"dp{world} (independent heads, no collective)",
+                   "l2": "flushed before every step (256 MiB write, outside the timed events)"},
+        "roofline": {"kernel": "fa_fwd_kernel<128, bf16 out, e4m3>", "bound": "tensor", "achieved": achieved,
+                     "peak": peak_tf, "unit": "TFLOP/s", "frac": achieved / peak_tf, "traffic": traffic,
+                     "peak_source": f"{peaks_src} {key} x {E4M3_PER_BF16} (nominal fp8/bf16 ratio)"},
+        "gpu_launches": args.steps,
+        "clocks": clocks.summary(),
+        "wall_s_timed_region": wall,
+        "e2e": e2e,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        fl, dt, n = oracle_sample_e4m3(w, causal, z, w.H, budget_s=args.cpu_budget)
+        result["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
+                                  "kind": "oracle",
+                                  "sample": f"{n} of {w.H} heads (b=0), fp64 forward on the dequantized inputs, "
+                                            f"{dt:.1f} s"}
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return result if rank == 0 else None
+
+
+def oracle_sample_e4m3(w, causal, z, heads, budget_s=None):
+    """The e4m3 oracle (fp64 attention on the dequantized bytes), head by head."""
+    import oracle.fp8
+    q8, k8, v8 = (z[n][0].numpy() for n in ("q", "k", "v"))
+    qd, kd, vd = (z[n][1] for n in ("q", "k", "v"))
+    done, t0 = 0, time.perf_counter()
+    for h in range(heads):
+        sl = (slice(0, 1), slice(None), slice(h, h + 1))
+        oracle.fp8.attention_forward_e4m3(q8[sl], k8[sl], v8[sl], qd, kd, vd, w.scale, causal)
+        done += 1
+        if budget_s is not None and time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return w.fwd_flops(causal) / (w.B * w.H) * done, dt, done
+
+
 # --------------------------------------------------------- reference arm
 def run_reference(args, w, causal):
     """The oracle as it stands, on the host cores: one head of the workload
-    (forward + backward, fp64) per step. Rank 0 only."""
+    (forward + backward, fp64; the e4m3 path: forward on the dequantized
+    inputs) per step. Rank 0 only."""
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if rank != 0:
         return None
+    if args.path == "fwd_e4m3":
+        return run_reference_e4m3(args, w, causal, world)
     inp64 = host_inputs64(w)
     for i in range(args.warmup):
         oracle_sample(w, causal, [a for a in inp64], 1)
@@ -374,6 +533,32 @@ def run_reference(args, w, causal):
     }
 
 
+def run_reference_e4m3(args, w, causal, world):
+    from exact_io_aware_96_b200.inputs import make_e4m3_inputs
+    z = make_e4m3_inputs(w)
+    for _ in range(args.warmup):
+        oracle_sample_e4m3(w, causal, z, 1)
+    t0 = time.perf_counter()
+    total = 0.0
+    for _ in range(args.steps):
+        fl, _, _ = oracle_sample_e4m3(w, causal, z, 1)
+        total += fl
+    dt = time.perf_counter() - t0
+    value = total / dt / 1e12
+    return {
+        "impl": "reference", "metric": METRIC_E4M3, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{w.name} shape, e4m3 inputs: B={w.B} H={w.H} S={w.S} D={w.D} causal={causal}; "
+                               "one head per step, forward only",
+                   "global_batch": w.B, "seq_len": w.S, "heads": 1, "head_dim": w.D, "causal": causal},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"one head of {w.name} per step (fp64 forward on dequantized e4m3 inputs)"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -381,6 +566,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="c4")
+    ap.add_argument("--path", choices=["fwd_bwd", "fwd_e4m3"], default="fwd_bwd",
+                    help="fwd_bwd: fa_fwd + fa_bwd in 16-bit (the default step); fwd_e4m3: fa_fwd_fp8 alone")
     ap.add_argument("--causal", type=int, choices=[0, 1], default=None,
                     help="override the workload's (first) mask setting")
     ap.add_argument("--no-e2e", action="store_true")
@@ -392,7 +579,12 @@ def main(argv=None):
     from exact_io_aware_96_b200.inputs import WORKLOADS
     w = WORKLOADS[args.workload]
     causal = bool(w.causal[0] if args.causal is None else args.causal)
-    res = run_reference(args, w, causal) if args.impl == "reference" else run_ours(args, w, causal)
+    if args.impl == "reference":
+        res = run_reference(args, w, causal)
+    elif args.path == "fwd_e4m3":
+        res = run_ours_fwd_e4m3(args, w, causal)
+    else:
+        res = run_ours(args, w, causal)
     if res is not None:
         print(json.dumps(res), flush=True)
 

@@ -131,6 +131,18 @@ def quantize_e4m3(x: torch.Tensor):
     return y.view(torch.uint8), descale
 
 
+def make_e4m3_inputs(w: Workload, B: int | None = None, seed: int | None = None):
+    """E4M3 inputs of workload ``w``'s shape: Q, K, V drawn as ``make_inputs``
+    draws them (fp32, same order and seed, Q and K times ``qk_std``), then
+    encoded by ``quantize_e4m3``. Returns {"q": (bytes, descale), "k": ..., "v": ...}."""
+    B = w.B if B is None else B
+    g = torch.Generator("cpu").manual_seed(w.seed if seed is None else seed)
+    out = {}
+    for name, std in (("q", w.qk_std), ("k", w.qk_std), ("v", 1.0)):
+        out[name] = quantize_e4m3(draw((B, w.S, w.H, w.D), g, torch.float32, std))
+    return out
+
+
 def sample_rows(S: int, block: int, n_random: int, seed: int):
     """Query rows checked at full size: tile edges, the middle, the tail, plus
     ``n_random`` rows drawn with ``seed``. Sorted, unique."""

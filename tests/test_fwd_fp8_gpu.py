@@ -7,7 +7,7 @@ import torch
 
 import oracle.fp8
 from exact_io_aware_96_b200 import fa
-from exact_io_aware_96_b200.inputs import WORKLOADS, make_inputs, quantize_e4m3, random_case, sample_rows
+from exact_io_aware_96_b200.inputs import WORKLOADS, make_e4m3_inputs, quantize_e4m3, random_case, sample_rows
 from tests.parity import check_fp8_o_lse, np64, run_fwd_fp8
 
 pytestmark = pytest.mark.gpu
@@ -108,9 +108,7 @@ def test_fp8_c4_full_size_sampled():
     """c4's shape (B1 H8 S8192 D128, causal) from c4's draws, quantized per
     tensor; O and LSE checked on sampled rows of every head."""
     w = WORKLOADS["c4"]
-    g = torch.Generator("cpu").manual_seed(w.seed)
-    c = {n: torch.randn((w.B, w.S, w.H, w.D), generator=g, dtype=torch.float32) for n in ("q", "k", "v")}
-    z = _quantized(c)
+    z = {n: (b, d, oracle.fp8.dequantize(b.numpy(), d)) for n, (b, d) in make_e4m3_inputs(w).items()}
     o, lse = run_fwd_fp8(z["q"][0].cuda(), z["k"][0].cuda(), z["v"][0].cuda(), z["q"][1], z["k"][1], z["v"][1],
                          True, w.scale)
     o, lse = np64(o), np64(lse)
