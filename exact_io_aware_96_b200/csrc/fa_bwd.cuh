@@ -32,17 +32,21 @@
 //   warp  12    TMA loader: K, V once; Q_i, dO_i, lse2_i, Dvec_i per query block
 //   warp  13    MMA issuer
 // Blocks are 128 keys x 128 queries. Tensor memory: dK and dV accumulators,
-// X (S^T, then 16-bit P^T and dS^T written back by the softmax warps and used
-// as the TMEM A operand of dV += P^T dO and dK += dS^T Q) and Y (dP^T, then
-// dQ^T = K^T dS^T (D = 128) or dQ = dS K (D = 64), with dS^T staged in
-// 128-byte swizzled smem). The MMA order per block i is dV(i), dK(i), dQ(i),
-// S^T(i+1), dP^T(i+1): S^T(i+1) runs while dQ(i) is drained out of Y, and the
-// softmax of block i+1 starts while dP^T(i+1) runs.
+// X (S^T, then 16-bit P^T written back by the softmax warps and used as the
+// TMEM A operand of dV += P^T dO) and Y (dP^T, then dQ^T = K^T dS^T (D = 128)
+// or dQ = dS K (D = 64)). dS^T goes to 128-byte swizzled smem, where it is
+// the A operand of dK += dS^T Q and an operand of the dQ product. The MMA
+// order per block i is dV(i), S^T(i+1), dK(i), dQ(i), dP^T(i+1): X is free as
+// soon as dV(i) has read P^T(i), so the softmax warps start on block i+1
+// while the tensor core runs dK(i) and dQ(i), and dP^T(i+1) follows once
+// dQ(i) has been drained out of Y.
 //
 // Page legend: [P1] "Miniconda-Python3.9环境下使用FlashAttention优化训练";
 // [P2] "使用FlashAttention优化PyTorch模型注意力计算"; [P4] the FlashAttention-2
 // walkthrough titled "企业官网建设流程全解析".
 #pragma once
+
+#include <type_traits>
 
 #include "fa.h"
 #include "fa_common.cuh"
@@ -152,16 +156,15 @@ struct BwdLayout {
   // requires (and checks) a 1024-aligned dynamic shared memory base.
   static constexpr int SMEM_ALLOC = (BYTES + 1024 <= SMEM_MAX) ? BYTES + 1024 : BYTES;
   static constexpr int TMEM_COLS = 512;
-  // TMEM columns: dK, dV accumulators; X holds S^T, then P^T and dS^T
-  // (16-bit); Y holds dP^T, then dQ.
+  // TMEM columns: dK, dV accumulators; X holds S^T, then P^T (16-bit); Y
+  // holds dP^T, then dQ.
   static constexpr int COL_DK = 0;
   static constexpr int COL_DV = D;
   static constexpr int COL_X = 2 * D;
   static constexpr int COL_Y = 2 * D + 128;
   // Softmax warpgroup g owns queries [64g, 64g + 64): it packs their P^T into
-  // X columns [64g, 64g + 32) and their dS^T into [64g + 32, 64g + 64).
+  // X columns [64g, 64g + 32).
   __host__ __device__ static constexpr int col_p(int kk) { return COL_X + (kk >> 2) * 64 + (kk & 3) * 8; }
-  __host__ __device__ static constexpr int col_ds(int kk) { return COL_X + (kk >> 2) * 64 + 32 + (kk & 3) * 8; }
 };
 
 template <int D, bool BF16>
@@ -252,114 +255,123 @@ __global__ void __launch_bounds__(448, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == kLoaderWarp) {
-    // ---------------------------------------------------------------- loader
-    if (lane == 0 && n > 0) {
-      mbar_arrive_expect_tx(kv_full, 2 * L::TILE);
-      for (int kb = 0; kb < L::KB; ++kb) {
-        tma_load_4d(smem + L::OFF_K + kb * L::BLK, &tmK, kv_full, kb * 64, n0, h, b);
-        tma_load_4d(smem + L::OFF_V + kb * L::BLK, &tmV, kv_full, kb * 64, n0, h, b);
-      }
-      int i = 0;
-      for (; i < n; ++i) {
-        const int st = i % QS;
-        const uint32_t ph = (i / QS) & 1;
-        if (!wait_bar(&q_empty[st], ph ^ 1, abort_flag, kRoleLoader, i)) break;
-        const int i0 = (i_start + i) * BM;
-        mbar_arrive_expect_tx(&q_full[st], 2 * L::TILE + 2 * BM * 4);
+  if (warp >= 12) {
+    if (warp == kLoaderWarp) {
+      // ---------------------------------------------------------------- loader
+      if (lane == 0 && n > 0) {
+        mbar_arrive_expect_tx(kv_full, 2 * L::TILE);
         for (int kb = 0; kb < L::KB; ++kb) {
-          tma_load_4d(smem + L::OFF_Q + st * L::TILE + kb * L::BLK, &tmQ, &q_full[st], kb * 64, i0, h, b);
-          tma_load_4d(smem + L::OFF_DO + st * L::TILE + kb * L::BLK, &tmdO, &q_full[st], kb * 64, i0, h, b);
+          tma_load_4d(smem + L::OFF_K + kb * L::BLK, &tmK, kv_full, kb * 64, n0, h, b);
+          tma_load_4d(smem + L::OFF_V + kb * L::BLK, &tmV, kv_full, kb * 64, n0, h, b);
         }
-        bulk_load(smem + L::OFF_LSE + st * BM * 4, a.lse2 + bh_row0 + i0, BM * 4, &q_full[st]);
-        bulk_load(smem + L::OFF_DVEC + st * BM * 4, a.dvec + bh_row0 + i0, BM * 4, &q_full[st]);
-      }
-      if (*abort_flag) {
-        drain_wait(kv_full, 0);
-        for (int j = max(0, i - QS); j < i; ++j) drain_wait(&q_full[j % QS], (j / QS) & 1);
-      }
-    }
-  } else if (warp == kMmaWarp) {
-    // ----------------------------------------------------------- MMA issuer
-    if (lane == 0 && n > 0) {
-      const uint32_t sK = smem_u32(smem + L::OFF_K);
-      const uint32_t sV = smem_u32(smem + L::OFF_V);
-      const uint32_t sQ = smem_u32(smem + L::OFF_Q);
-      const uint32_t sdO = smem_u32(smem + L::OFF_DO);
-      const uint32_t sDS = smem_u32(smem + L::OFF_DS);
-      // S^T = K Q^T, dP^T = V dO^T: M = 128 keys, N = 128 queries, K = D (both K-major).
-      const uint32_t id_s = idesc_f16(BF16, 128, 128, 0, 0);
-      // dV += P^T dO, dK += dS^T Q: M = 128 keys, N = D, K = 128 queries; A in TMEM, B MN-major.
-      const uint32_t id_kv = idesc_f16(BF16, 128, D, 0, 1);
-      // D = 128: dQ^T = K^T dS^T, M = head_dim, N = 128 queries, K = 128 keys; A = K viewed
-      // MN-major, B = dS^T MN-major. D = 64: dQ = dS K, M = 128 queries, N = D; A = dS^T
-      // viewed MN-major, B = K MN-major.
-      const uint32_t id_q = L::DQ_T ? idesc_f16(BF16, 128, 128, 1, 1) : idesc_f16(BF16, 128, D, 1, 1);
-      auto issue_kt = [&](uint32_t dcol, uint32_t kv, uint32_t qa) {  // dcol = kv-tile x qa-tile^T
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t o = (kk >> 2) * L::BLK + (kk & 3) * 32;
-          mma_ss(tmem + dcol, desc_sw128(kv + o, 16, 1024), desc_sw128(qa + o, 16, 1024), id_s, kk > 0);
+        int i = 0;
+        for (; i < n; ++i) {
+          const int st = i % QS;
+          const uint32_t ph = (i / QS) & 1;
+          if (!wait_bar(&q_empty[st], ph ^ 1, abort_flag, kRoleLoader, i)) break;
+          const int i0 = (i_start + i) * BM;
+          mbar_arrive_expect_tx(&q_full[st], 2 * L::TILE + 2 * BM * 4);
+          for (int kb = 0; kb < L::KB; ++kb) {
+            tma_load_4d(smem + L::OFF_Q + st * L::TILE + kb * L::BLK, &tmQ, &q_full[st], kb * 64, i0, h, b);
+            tma_load_4d(smem + L::OFF_DO + st * L::TILE + kb * L::BLK, &tmdO, &q_full[st], kb * 64, i0, h, b);
+          }
+          bulk_load(smem + L::OFF_LSE + st * BM * 4, a.lse2 + bh_row0 + i0, BM * 4, &q_full[st]);
+          bulk_load(smem + L::OFF_DVEC + st * BM * 4, a.dvec + bh_row0 + i0, BM * 4, &q_full[st]);
         }
-      };
-      bool ok = wait_bar(kv_full, 0, abort_flag, kRoleMma, -1) && wait_bar(&q_full[0], 0, abort_flag, kRoleMma, 0);
-      if (ok) {
-        tc_fence_after();
-        issue_kt(L::COL_X, sK, sQ);
-        mma_commit(sx_full);
-        issue_kt(L::COL_Y, sV, sdO);
-        mma_commit(dp_full);
-      }
-      for (int i = 0; ok && i < n; ++i) {
-        const int st = i % QS;
-        const uint32_t ph = i & 1;
-        const uint32_t qa = sQ + st * L::TILE;
-        const uint32_t da = sdO + st * L::TILE;
-        if (!(ok = wait_bar(p_ready, ph, abort_flag, kRoleMma, i))) break;
-        tc_fence_after();
-        // dV += P^T dO
-#pragma unroll
-        for (int kk = 0; kk < BM / 16; ++kk)
-          mma_ts(tmem + L::COL_DV, tmem + L::col_p(kk), desc_sw128(da + kk * 2048, L::BLK, 1024), id_kv,
-                 (i > 0 || kk > 0) ? 1u : 0u);
-        if (!(ok = wait_bar(ds_ready, ph, abort_flag, kRoleMma, i))) break;
-        tc_fence_after();
-        // dK += dS^T Q
-#pragma unroll
-        for (int kk = 0; kk < BM / 16; ++kk)
-          mma_ts(tmem + L::COL_DK, tmem + L::col_ds(kk), desc_sw128(qa + kk * 2048, L::BLK, 1024), id_kv,
-                 (i > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&q_empty[st]);
-        // dQ (or dQ^T) into Y: dP^T(i) there has been read by the softmax warps.
-#pragma unroll
-        for (int kk = 0; kk < L::BN / 16; ++kk) {
-          const uint64_t dk_desc = desc_sw128(sDS + kk * 2048, L::BLK, 1024);
-          const uint64_t k_desc = desc_sw128(sK + kk * 2048, L::BLK, 1024);
-          if constexpr (L::DQ_T)
-            mma_ss(tmem + L::COL_Y, k_desc, dk_desc, id_q, kk > 0);
-          else
-            mma_ss(tmem + L::COL_Y, dk_desc, k_desc, id_q, kk > 0);
+        if (*abort_flag) {
+          drain_wait(kv_full, 0);
+          for (int j = max(0, i - QS); j < i; ++j) drain_wait(&q_full[j % QS], (j / QS) & 1);
         }
-        mma_commit(dq_full);
-        mma_commit(ds_free);
-        if (i + 1 < n) {
-          // S^T(i+1) into X (after the MMAs that read P^T, dS^T from X); it
-          // runs while the dQ block is drained out of Y.
-          const int sn = (i + 1) % QS;
-          if (!(ok = wait_bar(&q_full[sn], ((i + 1) / QS) & 1, abort_flag, kRoleMma, i + 1))) break;
+      }
+    } else if (warp == kMmaWarp) {
+      // ----------------------------------------------------------- MMA issuer
+      if (lane == 0 && n > 0) {
+        const uint32_t sK = smem_u32(smem + L::OFF_K);
+        const uint32_t sV = smem_u32(smem + L::OFF_V);
+        const uint32_t sQ = smem_u32(smem + L::OFF_Q);
+        const uint32_t sdO = smem_u32(smem + L::OFF_DO);
+        const uint32_t sDS = smem_u32(smem + L::OFF_DS);
+        // S^T = K Q^T, dP^T = V dO^T: M = 128 keys, N = 128 queries, K = D (both K-major).
+        const uint32_t id_s = idesc_f16(BF16, 128, 128, 0, 0);
+        // dV += P^T dO, dK += dS^T Q: M = 128 keys, N = D, K = 128 queries; A in TMEM, B MN-major.
+        const uint32_t id_kv = idesc_f16(BF16, 128, D, 0, 1);
+        // D = 128: dQ^T = K^T dS^T, M = head_dim, N = 128 queries, K = 128 keys; A = K viewed
+        // MN-major, B = dS^T MN-major. D = 64: dQ = dS K, M = 128 queries, N = D; A = dS^T
+        // viewed MN-major, B = K MN-major.
+        const uint32_t id_q = L::DQ_T ? idesc_f16(BF16, 128, 128, 1, 1) : idesc_f16(BF16, 128, D, 1, 1);
+        auto issue_kt = [&](uint32_t dcol, uint32_t kv, uint32_t qa) {  // dcol = kv-tile x qa-tile^T
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t o = (kk >> 2) * L::BLK + (kk & 3) * 32;
+            mma_ss(tmem + dcol, desc_sw128(kv + o, 16, 1024), desc_sw128(qa + o, 16, 1024), id_s, kk > 0);
+          }
+        };
+        bool ok = wait_bar(kv_full, 0, abort_flag, kRoleMma, -1) && wait_bar(&q_full[0], 0, abort_flag, kRoleMma, 0);
+        if (ok) {
           tc_fence_after();
-          issue_kt(L::COL_X, sK, sQ + sn * L::TILE);
+          issue_kt(L::COL_X, sK, sQ);
           mma_commit(sx_full);
-          // dP^T(i+1) into Y once dQ(i) has been read out of it.
-          if (!(ok = wait_bar(dq_free, ph, abort_flag, kRoleMma, i))) break;
-          tc_fence_after();
-          issue_kt(L::COL_Y, sV, sdO + sn * L::TILE);
+          issue_kt(L::COL_Y, sV, sdO);
           mma_commit(dp_full);
         }
+        for (int i = 0; ok && i < n; ++i) {
+          const int st = i % QS;
+          const uint32_t ph = i & 1;
+          const uint32_t qa = sQ + st * L::TILE;
+          const uint32_t da = sdO + st * L::TILE;
+          if (!(ok = wait_bar(p_ready, ph, abort_flag, kRoleMma, i))) break;
+          tc_fence_after();
+          // dV += P^T dO
+#pragma unroll
+          for (int kk = 0; kk < BM / 16; ++kk)
+            mma_ts(tmem + L::COL_DV, tmem + L::col_p(kk), desc_sw128(da + kk * 2048, L::BLK, 1024), id_kv,
+                   (i > 0 || kk > 0) ? 1u : 0u);
+          if (i + 1 < n) {
+            // S^T(i+1) into X as soon as dV(i) has been issued: X held only
+            // P^T(i), which dV(i) reads first (the tensor pipe runs in issue
+            // order). The softmax of block i+1 then overlaps dK(i) and dQ(i).
+            const int sn = (i + 1) % QS;
+            if (!(ok = wait_bar(&q_full[sn], ((i + 1) / QS) & 1, abort_flag, kRoleMma, i + 1))) break;
+            tc_fence_after();
+            issue_kt(L::COL_X, sK, sQ + sn * L::TILE);
+            mma_commit(sx_full);
+          }
+          if (!(ok = wait_bar(ds_ready, ph, abort_flag, kRoleMma, i))) break;
+          tc_fence_after();
+          // dQ (or dQ^T) into Y first, so that its drain overlaps dK(i): dP^T(i)
+          // there has been read by the softmax warps.
+#pragma unroll
+          for (int kk = 0; kk < L::BN / 16; ++kk) {
+            const uint64_t dk_desc = desc_sw128(sDS + kk * 2048, L::BLK, 1024);
+            const uint64_t k_desc = desc_sw128(sK + kk * 2048, L::BLK, 1024);
+            if constexpr (L::DQ_T)
+              mma_ss(tmem + L::COL_Y, k_desc, dk_desc, id_q, kk > 0);
+            else
+              mma_ss(tmem + L::COL_Y, dk_desc, k_desc, id_q, kk > 0);
+          }
+          mma_commit(dq_full);
+          // dK += dS^T Q, dS^T from shared memory (K-major: 128 keys x 128 queries)
+#pragma unroll
+          for (int kk = 0; kk < BM / 16; ++kk) {
+            const uint32_t o = (kk >> 2) * L::BLK + (kk & 3) * 32;
+            mma_ss(tmem + L::COL_DK, desc_sw128(sDS + o, 16, 1024), desc_sw128(qa + kk * 2048, L::BLK, 1024), id_kv,
+                   (i > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&q_empty[st]);
+          mma_commit(ds_free);
+          if (i + 1 < n) {
+            // dP^T(i+1) into Y once dQ(i) has been read out of it.
+            const int sn = (i + 1) % QS;
+            if (!(ok = wait_bar(dq_free, ph, abort_flag, kRoleMma, i))) break;
+            tc_fence_after();
+            issue_kt(L::COL_Y, sV, sdO + sn * L::TILE);
+            mma_commit(dp_full);
+          }
+        }
+        mma_commit(mma_done);
+        mma_commit(drain);
+        drain_wait(drain, 0);
       }
-      mma_commit(mma_done);
-      mma_commit(drain);
-      drain_wait(drain, 0);
     }
   } else if (warp < 8) {
     // --------------- P^T and dS^T: one key row per thread, 64 query columns per warpgroup
@@ -391,34 +403,57 @@ __global__ void __launch_bounds__(448, 1)
         uint32_t sv[2][32];
         tmem_ld32(tX, sv[0]);
         tmem_ld32(tX + 32, sv[1]);
-        float4 lv[16];  // lse2 of this warpgroup's 64 queries, loaded while the TMEM load is in flight
-#pragma unroll
-        for (int u = 0; u < 16; ++u) lv[u] = reinterpret_cast<const float4*>(lse_s)[u];
         tmem_ld_wait();
         reg_fence(sv[0]);
         reg_fence(sv[1]);
+        // Blocks with a masked entry in this warp (causal diagonal, key tail,
+        // query rows with no key) take the MUFU exp2 everywhere, so that masked
+        // entries give exact zeros. Other blocks send one pair in four through
+        // the polynomial exp2 on the FMA pipe.
+        auto block = [&](auto masked) {
+          const uint64_t sl2x2 = f2(sl2, sl2);
 #pragma unroll
-        for (int c = 0; c < 2; ++c)
+          for (int c = 0; c < 2; ++c) {
+            float4 lv[8];  // lse2 of these 32 queries
 #pragma unroll
-          for (int e = 0; e < 32; e += 4) {
-            const int q = 32 * c + e;
-            const float4 L4 = lv[q >> 2];
-            float s0 = __uint_as_float(sv[c][e]), s1 = __uint_as_float(sv[c][e + 1]);
-            float s2 = __uint_as_float(sv[c][e + 2]), s3 = __uint_as_float(sv[c][e + 3]);
-            s0 = (q < cm) ? -INFINITY : s0;
-            s1 = (q + 1 < cm) ? -INFINITY : s1;
-            s2 = (q + 2 < cm) ? -INFINITY : s2;
-            s3 = (q + 3 < cm) ? -INFINITY : s3;
-            pp[c][e >> 1] = pack2<BF16>(ex2(fmaf(s0, sl2, -L4.x)), ex2(fmaf(s1, sl2, -L4.y)));
-            pp[c][(e >> 1) + 1] = pack2<BF16>(ex2(fmaf(s2, sl2, -L4.z)), ex2(fmaf(s3, sl2, -L4.w)));
+            for (int u = 0; u < 8; ++u) lv[u] = reinterpret_cast<const float4*>(lse_s + 32 * c)[u];
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              const int q = 32 * c + e;
+              const float4 L4 = lv[e >> 2];
+              float s0 = __uint_as_float(sv[c][e]), s1 = __uint_as_float(sv[c][e + 1]);
+              const float l0 = (e & 2) ? L4.z : L4.x, l1 = (e & 2) ? L4.w : L4.y;
+              if constexpr (decltype(masked)::value) {
+                s0 = (q < cm) ? -INFINITY : s0;
+                s1 = (q + 1 < cm) ? -INFINITY : s1;
+                pp[c][e >> 1] = pack2<BF16>(ex2(fmaf(s0, sl2, -l0)), ex2(fmaf(s1, sl2, -l1)));
+              } else {
+                const uint64_t t = fma2(f2(s0, s1), sl2x2, f2(-l0, -l1));
+                float p0, p1;
+                if (((e >> 1) & 3) == 3) {
+                  f2_split(exp2_poly2(t), p0, p1);
+                } else {
+                  f2_split(t, p0, p1);
+                  p0 = ex2(p0);
+                  p1 = ex2(p1);
+                }
+                pp[c][e >> 1] = pack2<BF16>(p0, p1);
+              }
+            }
           }
+        };
+        if (__any_sync(0xffffffffu, cm > 0))
+          block(std::true_type{});
+        else
+          block(std::false_type{});
       }
       tmem_st16(tX, pp[0]);       // X columns [64g, 64g + 32): read above
       tmem_st16(tX + 16, pp[1]);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(p_ready);
-      // Phase B: dS^T = P^T (dP^T - Dvec) -> 16-bit pairs into X and into smem.
+      // Phase B: dS^T = P^T (dP^T - Dvec) -> 16-bit pairs into swizzled smem
+      // (the A operand of dK, the B operand of dQ^T / A of dQ).
       ok = __all_sync(0xffffffffu, wait_bar(dp_full, ph, abort_flag, kRoleSoftmax, i) &&
                                        wait_bar(ds_free, ph ^ 1, abort_flag, kRoleSoftmax, i));
       if (!ok) break;
@@ -443,7 +478,6 @@ __global__ void __launch_bounds__(448, 1)
           dsp[(e >> 1) + 1] =
               pack2<BF16>(pb.x * (__uint_as_float(dpv[e + 2]) - V4.z), pb.y * (__uint_as_float(dpv[e + 3]) - V4.w));
         }
-        tmem_st16(tX + 32 + 16 * c, dsp);  // X columns [64g + 32, 64g + 64): read in phase A
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const int chunk = 4 * c + u;
@@ -451,7 +485,6 @@ __global__ void __launch_bounds__(448, 1)
                        dsp[4 * u + 3]);
         }
       }
-      tmem_st_wait();
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(ds_ready);
@@ -505,39 +538,47 @@ __global__ void __launch_bounds__(448, 1)
       const int64_t row0 = bh_row0 + (i_start + i) * BM;
       if constexpr (L::DQ_T) {
         // lane = head_dim index d, columns = 128 query rows: for each query the
-        // warp adds 32 consecutive floats (one 128-byte line).
+        // warp adds 32 consecutive floats (one 128-byte line). Three quarters
+        // of the block are read before any reduction is issued and the last
+        // quarter after the first quarter's reductions, so that Y is released
+        // (and dP^T(i+1) may start) after 32 of the 128 reductions.
         float* col = a.dq_acc + row0 * D + tr;
+        uint32_t v[3][32];
 #pragma unroll
-        for (int part = 0; part < 4; ++part) {
-          uint32_t v[32];
-          tmem_ld32(tY + 32 * part, v);
-          tmem_ld_wait();
-          reg_fence(v);
-          if (part == 3) {
-            tc_fence_before();
-            mbar_arrive(dq_free);  // Y may take dP^T(i+1) now
-          }
+        for (int part = 0; part < 3; ++part) tmem_ld32(tY + 32 * part, v[part]);
+        tmem_ld_wait();
 #pragma unroll
-          for (int c = 0; c < 32; ++c) red_add_f32(col + (32 * part + c) * D, __uint_as_float(v[c]));
-        }
+        for (int part = 0; part < 3; ++part) reg_fence(v[part]);
+#pragma unroll
+        for (int c = 0; c < 32; ++c) red_add_f32(col + c * D, __uint_as_float(v[0][c]));
+        tmem_ld32(tY + 96, v[0]);
+        tmem_ld_wait();
+        reg_fence(v[0]);
+        tc_fence_before();
+        mbar_arrive(dq_free);  // Y may take dP^T(i+1) now
+#pragma unroll
+        for (int part = 1; part < 4; ++part)
+#pragma unroll
+          for (int c = 0; c < 32; ++c)
+            red_add_f32(col + (32 * part + c) * D, __uint_as_float(v[part == 3 ? 0 : part][c]));
       } else {
-        // lane = query row, columns = head_dim (64).
+        // lane = query row, columns = head_dim (64): the whole block fits in
+        // registers, so Y is released before the reductions.
         float* row = a.dq_acc + (row0 + tr) * D;
+        uint32_t v[D / 32][32];
 #pragma unroll
-        for (int part = 0; part < D / 32; ++part) {
-          uint32_t v[32];
-          tmem_ld32(tY + 32 * part, v);
-          tmem_ld_wait();
-          reg_fence(v);
-          if (part == D / 32 - 1) {
-            tc_fence_before();
-            mbar_arrive(dq_free);
-          }
+        for (int part = 0; part < D / 32; ++part) tmem_ld32(tY + 32 * part, v[part]);
+        tmem_ld_wait();
+#pragma unroll
+        for (int part = 0; part < D / 32; ++part) reg_fence(v[part]);
+        tc_fence_before();
+        mbar_arrive(dq_free);
+#pragma unroll
+        for (int part = 0; part < D / 32; ++part)
 #pragma unroll
           for (int c = 0; c < 32; c += 4)
-            red_add_v4_f32(row + 32 * part + c, __uint_as_float(v[c]), __uint_as_float(v[c + 1]),
-                           __uint_as_float(v[c + 2]), __uint_as_float(v[c + 3]));
-        }
+            red_add_v4_f32(row + 32 * part + c, __uint_as_float(v[part][c]), __uint_as_float(v[part][c + 1]),
+                           __uint_as_float(v[part][c + 2]), __uint_as_float(v[part][c + 3]));
       }
     }
   }
