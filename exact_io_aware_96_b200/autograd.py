@@ -28,18 +28,19 @@ def _kernel_ready(t: torch.Tensor) -> torch.Tensor:
 
 class FlashAttentionFunction(torch.autograd.Function):
     @staticmethod
-    def forward(ctx, q, k, v, causal: bool, scale):
+    def forward(ctx, q, k, v, causal: bool, scale, deterministic: bool = False):
         q, k, v = _kernel_ready(q), _kernel_ready(k), _kernel_ready(v)
         o, lse = fa.forward(q, k, v, causal=causal, scale=scale)
         ctx.save_for_backward(q, k, v, o, lse)
-        ctx.causal, ctx.scale = causal, scale
+        ctx.causal, ctx.scale, ctx.deterministic = causal, scale, deterministic
         return o
 
     @staticmethod
     def backward(ctx, do):
         q, k, v, o, lse = ctx.saved_tensors
-        dq, dk, dv = fa.backward(q, k, v, o, lse, _kernel_ready(do), causal=ctx.causal, scale=ctx.scale)
-        return dq, dk, dv, None, None
+        dq, dk, dv = fa.backward(q, k, v, o, lse, _kernel_ready(do), causal=ctx.causal, scale=ctx.scale,
+                                 deterministic=ctx.deterministic)
+        return dq, dk, dv, None, None, None
 
 
 class FlashAttentionQKVPackedFunction(torch.autograd.Function):
@@ -69,10 +70,11 @@ def _kernel_ready_packed(qkv: torch.Tensor) -> torch.Tensor:
     return qkv if ok else qkv.contiguous()
 
 
-def flash_attn_func(q, k, v, causal: bool = False, softmax_scale=None):
-    """O = softmax(scale q k^T [+ causal mask]) v on [B, S, H, D] CUDA tensors, differentiable."""
+def flash_attn_func(q, k, v, causal: bool = False, softmax_scale=None, deterministic: bool = False):
+    """O = softmax(scale q k^T [+ causal mask]) v on [B, S, H, D] CUDA tensors, differentiable.
+    ``deterministic=True`` makes the backward's dq bit-reproducible."""
     scale = q.shape[-1] ** -0.5 if softmax_scale is None else float(softmax_scale)
-    return FlashAttentionFunction.apply(q, k, v, bool(causal), scale)
+    return FlashAttentionFunction.apply(q, k, v, bool(causal), scale, bool(deterministic))
 
 
 def flash_attn_qkvpacked_func(qkv, causal: bool = False, softmax_scale=None):

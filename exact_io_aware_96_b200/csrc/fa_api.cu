@@ -166,6 +166,14 @@ int launch_fwd_fp8(const fa_fwd_fp8_params* p, cudaStream_t stream) {
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+// Byte offset of the deterministic-mode dQ slots in the workspace: after the
+// fp32 accumulator, Dvec and base-2 LSE, rounded up to 256 bytes.
+uint64_t det_part_offset(int B, int H, int Sq, int D) {
+  const uint64_t dpad = D <= 64 ? 64 : 128;
+  const uint64_t rows = uint64_t(B) * H * ((uint64_t(Sq) + 127) / 128 * 128);
+  return (rows * (dpad + 2) * 4 + 255) / 256 * 256;
+}
+
 template <int D, bool BF16>
 int launch_bwd(const fa_bwd_params* p, cudaStream_t stream) {
   using L = fa::BwdLayout<D>;
@@ -192,6 +200,11 @@ int launch_bwd(const fa_bwd_params* p, cudaStream_t stream) {
   a.dq_acc = static_cast<float*>(p->workspace);
   a.dvec = a.dq_acc + rows * D;
   a.lse2 = a.dvec + rows;
+  a.nqb = (p->Sq + 127) / 128;
+  a.nkb = (p->Sk + 127) / 128;
+  a.dq_part = p->deterministic ? reinterpret_cast<float*>(static_cast<char*>(p->workspace) +
+                                                          det_part_offset(p->B, p->H, p->Sq, p->D))
+                               : nullptr;
   a.o_sb = p->o.stride_b, a.o_ss = p->o.stride_s, a.o_sh = p->o.stride_h;
   a.do_sb = p->dO.stride_b, a.do_ss = p->dO.stride_s, a.do_sh = p->dO.stride_h;
   a.dq_sb = p->dq.stride_b, a.dq_ss = p->dq.stride_s, a.dq_sh = p->dq.stride_h;
@@ -213,7 +226,10 @@ int launch_bwd(const fa_bwd_params* p, cudaStream_t stream) {
   kern<<<grid, L::kThreads, L::SMEM_ALLOC, stream>>>(mq, mk, mv, mdo, a);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   const int64_t dq_threads = int64_t(p->B) * p->H * p->Sq * G;
-  fa::fa_bwd_dq<D, BF16><<<unsigned((dq_threads + 255) / 256), 256, 0, stream>>>(a);
+  if (a.dq_part != nullptr)
+    fa::fa_bwd_dq_sum<D, BF16><<<unsigned((dq_threads + 255) / 256), 256, 0, stream>>>(a);
+  else
+    fa::fa_bwd_dq<D, BF16><<<unsigned((dq_threads + 255) / 256), 256, 0, stream>>>(a);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -250,7 +266,7 @@ int noalloc_scratch(void** out) {
 
 extern "C" {
 
-int fa_version(void) { return 100; }
+int fa_version(void) { return 200; }
 
 const char* fa_strerror(int s) {
   switch (s) {
@@ -358,6 +374,18 @@ size_t fa_bwd_workspace_size(int B, int H, int Sq, int D) {
   return size_t(bytes);
 }
 
+size_t fa_bwd_workspace_size_ex(int B, int H, int Sq, int Sk, int D, int deterministic) {
+  if (deterministic != 0 && deterministic != 1) return 0;
+  if (Sk < 1) return 0;
+  const size_t base = fa_bwd_workspace_size(B, H, Sq, D);
+  if (base == 0 || !deterministic) return base;
+  const uint64_t dpad = D <= 64 ? 64 : 128;
+  const uint64_t slots = uint64_t(B) * H * ((uint64_t(Sq) + 127) / 128) * ((uint64_t(Sk) + 127) / 128);
+  const uint64_t bytes = det_part_offset(B, H, Sq, D) + slots * 128 * dpad * 4;
+  if (bytes > (uint64_t(1) << 50)) return 0;
+  return size_t(bytes);
+}
+
 int fa_bwd_ex(const fa_bwd_params* p, fa_stream_t stream) {
   if (p == nullptr) return FA_ERR_INVALID_ARG;
   int st = check_common(p->B, p->H, p->Sq, p->Sk, p->D, p->scale, p->causal, p->dtype);
@@ -367,7 +395,8 @@ int fa_bwd_ex(const fa_bwd_params* p, fa_stream_t stream) {
     if ((st = check_view(*v)) != FA_OK) return st;
   if (p->lse == nullptr) return FA_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(p->lse) & 3u) return FA_ERR_MISALIGNED;
-  const size_t need = fa_bwd_workspace_size(p->B, p->H, p->Sq, p->D);
+  if (p->deterministic != 0 && p->deterministic != 1) return FA_ERR_INVALID_ARG;
+  const size_t need = fa_bwd_workspace_size_ex(p->B, p->H, p->Sq, p->Sk, p->D, p->deterministic);
   if (p->workspace == nullptr || p->workspace_bytes < need || need == 0) return FA_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(p->workspace) & 255u) return FA_ERR_MISALIGNED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

@@ -85,9 +85,11 @@ __global__ void __launch_bounds__(256) fa_bwd_pre(const BwdArgs a) {
   }
 #pragma unroll
   for (int s = G / 2; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
-  float4* dq = reinterpret_cast<float4*>(a.dq_acc + row * D + part * 8);
-  dq[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-  dq[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (a.dq_part == nullptr) {  // the atomic accumulator starts from zero
+    float4* dq = reinterpret_cast<float4*>(a.dq_acc + row * D + part * 8);
+    dq[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    dq[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
   if (part == 0) {
     a.dvec[row] = acc;
     float l2 = INFINITY;
@@ -120,6 +122,44 @@ __global__ void __launch_bounds__(256) fa_bwd_dq(const BwdArgs a) {
   out.y = sm100::pack2<BF16>(x.z * s, x.w * s);
   out.z = sm100::pack2<BF16>(y.x * s, y.y * s);
   out.w = sm100::pack2<BF16>(y.z * s, y.w * s);
+  *reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(a.dq) + b * a.dq_sb + static_cast<int64_t>(i) * a.dq_ss +
+                            h * a.dq_sh + part * 8) = out;
+}
+
+// ------------------------------------------------ deterministic dq reduction
+// dq = scale * sum over key blocks, in increasing key-block order, of the
+// dQ blocks the main kernel stored in their (query block, key block) slots.
+// A key block contributes to query block qb iff qb >= bwd_first_qblock(kvb),
+// which is where the main kernel starts its query loop. One group of 8
+// columns per thread, as fa_bwd_dq.
+template <int D, bool BF16>
+__global__ void __launch_bounds__(256) fa_bwd_dq_sum(const BwdArgs a) {
+  constexpr int G = D / 8;
+  const int64_t gid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t row = gid / G;  // (b, h, i) with i < Sq
+  const int part = static_cast<int>(gid % G);
+  if (row >= static_cast<int64_t>(a.B) * a.H * a.Sq || part * 8 >= a.d) return;
+  const int i = static_cast<int>(row % a.Sq);
+  const int bh = static_cast<int>(row / a.Sq);
+  const int h = bh % a.H;
+  const int b = bh / a.H;
+  const int qb = i / 128;
+  const float* slot = a.dq_part + (static_cast<int64_t>(bh) * a.nqb + qb) * a.nkb * (128 * D) +
+                      (i % 128) * D + part * 8;
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  for (int kvb = 0; kvb < a.nkb; ++kvb) {
+    if (qb < bwd_first_qblock(kvb, a.Sq, a.Sk, a.causal)) break;  // later key blocks start later still
+    const float4* src = reinterpret_cast<const float4*>(slot + static_cast<int64_t>(kvb) * (128 * D));
+    const float4 x = src[0], y = src[1];
+    acc[0] += x.x, acc[1] += x.y, acc[2] += x.z, acc[3] += x.w;
+    acc[4] += y.x, acc[5] += y.y, acc[6] += y.z, acc[7] += y.w;
+  }
+  const float s = a.scale;
+  uint4 out;
+  out.x = sm100::pack2<BF16>(acc[0] * s, acc[1] * s);
+  out.y = sm100::pack2<BF16>(acc[2] * s, acc[3] * s);
+  out.z = sm100::pack2<BF16>(acc[4] * s, acc[5] * s);
+  out.w = sm100::pack2<BF16>(acc[6] * s, acc[7] * s);
   *reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(a.dq) + b * a.dq_sb + static_cast<int64_t>(i) * a.dq_ss +
                             h * a.dq_sh + part * 8) = out;
 }
@@ -214,11 +254,7 @@ __global__ void __launch_bounds__(448, 1)
   const int n0 = kvb * L::BN;
   const int off = a.Sk - a.Sq;
   const int nqb = (a.Sq + BM - 1) / BM;
-  int i_start = 0;
-  if (a.causal) {
-    const int qmin = n0 - off;  // smallest query row that may see key n0
-    i_start = qmin <= 0 ? 0 : qmin / BM;
-  }
+  const int i_start = bwd_first_qblock(kvb, a.Sq, a.Sk, a.causal);
   const int n = max(0, nqb - i_start);
   const int64_t bh_row0 = static_cast<int64_t>(b * a.H + h) * a.Sq_pad;
 
@@ -531,56 +567,78 @@ __global__ void __launch_bounds__(448, 1)
     // ------------------------------------------------- dQ drain (warps 8-11)
     const int tr = (warp & 3) * 32 + lane;  // TMEM lane
     const uint32_t tY = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16) + L::COL_Y;
-    for (int i = 0; i < n; ++i) {
-      const bool ok = __all_sync(0xffffffffu, wait_bar(dq_full, i & 1, abort_flag, kRoleSoftmax, i));
-      if (!ok) break;
-      tc_fence_after();
-      const int64_t row0 = bh_row0 + (i_start + i) * BM;
-      if constexpr (L::DQ_T) {
-        // lane = head_dim index d, columns = 128 query rows: for each query the
-        // warp adds 32 consecutive floats (one 128-byte line). Three quarters
-        // of the block are read before any reduction is issued and the last
-        // quarter after the first quarter's reductions, so that Y is released
-        // (and dP^T(i+1) may start) after 32 of the 128 reductions.
-        float* col = a.dq_acc + row0 * D + tr;
-        uint32_t v[3][32];
+    // DET: store the block into its own slot (deterministic mode) instead of
+    // adding it into the shared accumulator.
+    auto drain = [&](auto det) {
+      constexpr bool DET = decltype(det)::value;
+      auto put = [&](float* p, float x) {
+        if constexpr (DET)
+          *p = x;
+        else
+          red_add_f32(p, x);
+      };
+      for (int i = 0; i < n; ++i) {
+        const bool ok = __all_sync(0xffffffffu, wait_bar(dq_full, i & 1, abort_flag, kRoleSoftmax, i));
+        if (!ok) break;
+        tc_fence_after();
+        const int qb = i_start + i;
+        // block base: row0 of the accumulator, or the (qb, kvb) slot
+        float* base = DET ? a.dq_part + ((static_cast<int64_t>(hb) * a.nqb + qb) * a.nkb + kvb) * (BM * D)
+                          : a.dq_acc + (bh_row0 + static_cast<int64_t>(qb) * BM) * D;
+        if constexpr (L::DQ_T) {
+          // lane = head_dim index d, columns = 128 query rows: for each query the
+          // warp writes 32 consecutive floats (one 128-byte line). Three quarters
+          // of the block are read before any write is issued and the last
+          // quarter after the first quarter's writes, so that Y is released
+          // (and dP^T(i+1) may start) after 32 of the 128 writes.
+          float* col = base + tr;
+          uint32_t v[3][32];
 #pragma unroll
-        for (int part = 0; part < 3; ++part) tmem_ld32(tY + 32 * part, v[part]);
-        tmem_ld_wait();
+          for (int part = 0; part < 3; ++part) tmem_ld32(tY + 32 * part, v[part]);
+          tmem_ld_wait();
 #pragma unroll
-        for (int part = 0; part < 3; ++part) reg_fence(v[part]);
+          for (int part = 0; part < 3; ++part) reg_fence(v[part]);
 #pragma unroll
-        for (int c = 0; c < 32; ++c) red_add_f32(col + c * D, __uint_as_float(v[0][c]));
-        tmem_ld32(tY + 96, v[0]);
-        tmem_ld_wait();
-        reg_fence(v[0]);
-        tc_fence_before();
-        mbar_arrive(dq_free);  // Y may take dP^T(i+1) now
+          for (int c = 0; c < 32; ++c) put(col + c * D, __uint_as_float(v[0][c]));
+          tmem_ld32(tY + 96, v[0]);
+          tmem_ld_wait();
+          reg_fence(v[0]);
+          tc_fence_before();
+          mbar_arrive(dq_free);  // Y may take dP^T(i+1) now
 #pragma unroll
-        for (int part = 1; part < 4; ++part)
+          for (int part = 1; part < 4; ++part)
 #pragma unroll
-          for (int c = 0; c < 32; ++c)
-            red_add_f32(col + (32 * part + c) * D, __uint_as_float(v[part == 3 ? 0 : part][c]));
-      } else {
-        // lane = query row, columns = head_dim (64): the whole block fits in
-        // registers, so Y is released before the reductions.
-        float* row = a.dq_acc + (row0 + tr) * D;
-        uint32_t v[D / 32][32];
+            for (int c = 0; c < 32; ++c) put(col + (32 * part + c) * D, __uint_as_float(v[part == 3 ? 0 : part][c]));
+        } else {
+          // lane = query row, columns = head_dim (64): the whole block fits in
+          // registers, so Y is released before the writes.
+          float* row = base + tr * D;
+          uint32_t v[D / 32][32];
 #pragma unroll
-        for (int part = 0; part < D / 32; ++part) tmem_ld32(tY + 32 * part, v[part]);
-        tmem_ld_wait();
+          for (int part = 0; part < D / 32; ++part) tmem_ld32(tY + 32 * part, v[part]);
+          tmem_ld_wait();
 #pragma unroll
-        for (int part = 0; part < D / 32; ++part) reg_fence(v[part]);
-        tc_fence_before();
-        mbar_arrive(dq_free);
+          for (int part = 0; part < D / 32; ++part) reg_fence(v[part]);
+          tc_fence_before();
+          mbar_arrive(dq_free);
 #pragma unroll
-        for (int part = 0; part < D / 32; ++part)
+          for (int part = 0; part < D / 32; ++part)
 #pragma unroll
-          for (int c = 0; c < 32; c += 4)
-            red_add_v4_f32(row + 32 * part + c, __uint_as_float(v[part][c]), __uint_as_float(v[part][c + 1]),
-                           __uint_as_float(v[part][c + 2]), __uint_as_float(v[part][c + 3]));
+            for (int c = 0; c < 32; c += 4) {
+              const float x0 = __uint_as_float(v[part][c]), x1 = __uint_as_float(v[part][c + 1]);
+              const float x2 = __uint_as_float(v[part][c + 2]), x3 = __uint_as_float(v[part][c + 3]);
+              if constexpr (DET)
+                *reinterpret_cast<float4*>(row + 32 * part + c) = make_float4(x0, x1, x2, x3);
+              else
+                red_add_v4_f32(row + 32 * part + c, x0, x1, x2, x3);
+            }
+        }
       }
-    }
+    };
+    if (a.dq_part != nullptr)
+      drain(std::true_type{});
+    else
+      drain(std::false_type{});
   }
 
   tc_fence_before();

@@ -70,6 +70,14 @@ struct FwdArgs {
   int n_qblocks;     // ceil(Sq / 256)
 };
 
+// First query block that key block kvb contributes to: with a causal mask,
+// the block holding the smallest query row i with kvb * 128 <= i + (Sk - Sq).
+__host__ __device__ inline int bwd_first_qblock(int kvb, int Sq, int Sk, int causal) {
+  if (!causal) return 0;
+  const int qmin = kvb * 128 - (Sk - Sq);
+  return qmin <= 0 ? 0 : qmin / 128;
+}
+
 struct BwdArgs {
   const void* o;
   const void* dO;
@@ -80,6 +88,12 @@ struct BwdArgs {
   float* dq_acc;  // fp32 [B, H, Sq_pad, D]
   float* dvec;    // fp32 [B, H, Sq_pad]: sum_d dO_id O_id
   float* lse2;    // fp32 [B, H, Sq_pad]: LSE * log2(e); +inf where no key or padding
+  // Deterministic mode (non-null): fp32 [B*H][nqb][nkb][128][D] slots, one per
+  // (query block, key block) pair; each key block stores its dQ block there
+  // and fa_bwd_dq_sum adds the slots in key-block order. Null: dQ blocks are
+  // added into dq_acc with atomics.
+  float* dq_part;
+  int nqb, nkb;   // ceil(Sq / 128), ceil(Sk / 128)
   int64_t o_sb, o_ss, o_sh;
   int64_t do_sb, do_ss, do_sh;
   int64_t dq_sb, dq_ss, dq_sh;

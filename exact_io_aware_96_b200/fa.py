@@ -24,7 +24,7 @@ STATUS = {
 }
 FA_NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 EXPORTED = ("fa_fwd", "fa_fwd_ex", "fa_fwd_fp8", "fa_fwd_fp8_ex", "fa_bwd", "fa_bwd_ex", "fa_bwd_noalloc",
-            "fa_bwd_workspace_size", "fa_last_device_status", "fa_strerror", "fa_version")
+            "fa_bwd_workspace_size", "fa_bwd_workspace_size_ex", "fa_last_device_status", "fa_strerror", "fa_version")
 
 
 class FaTensor(ctypes.Structure):
@@ -56,7 +56,7 @@ class BwdParams(ctypes.Structure):
                 ("B", ctypes.c_int), ("H", ctypes.c_int), ("Sq", ctypes.c_int), ("Sk", ctypes.c_int),
                 ("D", ctypes.c_int), ("scale", ctypes.c_float), ("causal", ctypes.c_int),
                 ("dtype", ctypes.c_int), ("workspace", ctypes.c_void_p),
-                ("workspace_bytes", ctypes.c_size_t)]
+                ("workspace_bytes", ctypes.c_size_t), ("deterministic", ctypes.c_int)]
 
 
 class FaError(RuntimeError):
@@ -92,6 +92,8 @@ def lib():
         L.fa_bwd_noalloc.restype = i
         L.fa_bwd_workspace_size.argtypes = [i, i, i, i]
         L.fa_bwd_workspace_size.restype = sz
+        L.fa_bwd_workspace_size_ex.argtypes = [i, i, i, i, i, i]
+        L.fa_bwd_workspace_size_ex.restype = sz
         L.fa_last_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
         L.fa_last_device_status.restype = i
         L.fa_strerror.argtypes = [i]
@@ -139,6 +141,10 @@ def fa_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, B, H, Sq, Sk, D, scale, caus
 
 def fa_bwd_workspace_size(B, H, Sq, D) -> int:
     return lib().fa_bwd_workspace_size(B, H, Sq, D)
+
+
+def fa_bwd_workspace_size_ex(B, H, Sq, Sk, D, deterministic) -> int:
+    return lib().fa_bwd_workspace_size_ex(B, H, Sq, Sk, D, deterministic)
 
 
 def fa_last_device_status():
@@ -233,14 +239,19 @@ def forward_fp8(q, k, v, q_descale, k_descale, v_descale, causal=False, scale=No
     return out, lse
 
 
-def workspace_for(B, H, Sq, D, device) -> torch.Tensor:
-    n = fa_bwd_workspace_size(B, H, Sq, D)
+def workspace_for(B, H, Sq, D, device, Sk=None, deterministic=False) -> torch.Tensor:
+    if deterministic:
+        n = fa_bwd_workspace_size_ex(B, H, Sq, Sq if Sk is None else Sk, D, 1)
+    else:
+        n = fa_bwd_workspace_size(B, H, Sq, D)
     return torch.empty(n, dtype=torch.uint8, device=device)
 
 
 def backward(q, k, v, o, lse, do, causal=False, scale=None, dq=None, dk=None, dv=None,
-             workspace=None, stream=None):
-    """dQ, dK, dV of L = sum(dO * O) for O = attention(q, k, v)."""
+             workspace=None, stream=None, deterministic=False):
+    """dQ, dK, dV of L = sum(dO * O) for O = attention(q, k, v).
+    ``deterministic=True`` sums dQ in a fixed order (bit-identical runs; more
+    workspace and time)."""
     B, Sq, H, D = q.shape
     Sk = k.shape[1]
     dt = _dtype_code(q)
@@ -250,10 +261,10 @@ def backward(q, k, v, o, lse, do, causal=False, scale=None, dq=None, dk=None, dv
     dk = torch.empty((B, Sk, H, D), dtype=q.dtype, device=q.device) if dk is None else dk
     dv = torch.empty((B, Sk, H, D), dtype=q.dtype, device=q.device) if dv is None else dv
     if workspace is None:
-        workspace = workspace_for(B, H, Sq, D, q.device)
+        workspace = workspace_for(B, H, Sq, D, q.device, Sk=Sk, deterministic=deterministic)
     p = BwdParams(_view(q), _view(k), _view(v), _view(o), _view(do), lse.data_ptr(),
                   _view(dq), _view(dk), _view(dv), B, H, Sq, Sk, D, float(scale),
-                  int(bool(causal)), dt, workspace.data_ptr(), workspace.numel())
+                  int(bool(causal)), dt, workspace.data_ptr(), workspace.numel(), int(bool(deterministic)))
     st = fa_bwd_ex(p, _stream(stream))
     if st != FA_OK:
         raise FaError(st, "fa_bwd_ex")

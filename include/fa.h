@@ -117,8 +117,15 @@ typedef struct {
   float scale;
   int causal;
   int dtype;
-  void* workspace; /* device scratch, >= fa_bwd_workspace_size(B, H, Sq, D) bytes, 256-byte aligned */
+  void* workspace; /* device scratch, >= fa_bwd_workspace_size_ex(B, H, Sq, Sk, D,
+                      deterministic) bytes, 256-byte aligned */
   size_t workspace_bytes;
+  int deterministic; /* 0: dq summed with fp32 atomics (fast; last bits may vary
+                        between runs). 1: every (query block, key block) dQ block
+                        is stored in its own workspace slot and the slots are
+                        added in key-block order by a last kernel, so dq, like
+                        dk and dv, is bit-identical from run to run. Anything
+                        else is FA_ERR_INVALID_ARG. */
 } fa_bwd_params;
 
 /* Forward ([P1] "性能引擎"; [P2] items 1-2; [P4] §3.1, §3.2).
@@ -189,7 +196,8 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o,
            int dtype, void* workspace, size_t workspace_bytes,
            fa_stream_t stream);
 
-/* Backward on strided views. Same semantics. */
+/* Backward on strided views. Same semantics, plus the deterministic mode
+   (fa_bwd_params.deterministic; the pages are silent on it). */
 int fa_bwd_ex(const fa_bwd_params* p, fa_stream_t stream);
 
 /* Backward that allocates nothing and takes no workspace. Not a method step:
@@ -228,6 +236,14 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
    Sq_pad is Sq rounded up to a multiple of 128 and Dk is the kernel width
    (64 for D <= 64, else 128). Returns 0 for sizes < 1 or on overflow. */
 size_t fa_bwd_workspace_size(int B, int H, int Sq, int D);
+
+/* Workspace of fa_bwd_ex for either mode. deterministic = 0 gives
+   fa_bwd_workspace_size(B, H, Sq, D). deterministic = 1 adds, after that
+   (rounded up to 256 bytes), one fp32 [128][Dk] slot per (b, h, query block,
+   key block): B*H*ceil(Sq/128)*ceil(Sk/128)*128*Dk*4 bytes (2.15 GB for
+   B*H = 8, Sq = Sk = 8192, D = 128). Returns 0 for sizes < 1, a flag other
+   than 0 or 1, or on overflow. */
+size_t fa_bwd_workspace_size_ex(int B, int H, int Sq, int Sk, int D, int deterministic);
 
 /* Synchronises the current device, returns the status word recorded by
    kernels since the last call (FA_OK or FA_ERR_TIMEOUT) and clears it.

@@ -44,6 +44,19 @@ def test_workspace_size(fa_lib):
     assert fa.fa_bwd_workspace_size(1, 1, -5, 64) == 0
 
 
+def test_workspace_size_ex(fa_lib):
+    # mode 0 is the plain size; mode 1 adds (rounded to 256 B) one fp32 [128][Dk] slot per block pair
+    assert fa.fa_bwd_workspace_size_ex(2, 12, 2000, 2000, 64, 0) == fa.fa_bwd_workspace_size(2, 12, 2000, 64)
+    base = fa.fa_bwd_workspace_size(1, 8, 8192, 128)
+    assert base % 256 == 0
+    assert fa.fa_bwd_workspace_size_ex(1, 8, 8192, 8192, 128, 1) == base + 8 * 64 * 64 * 128 * 128 * 4
+    base = fa.fa_bwd_workspace_size(2, 3, 129, 32)   # not a multiple of 256: rounded up
+    off = (base + 255) // 256 * 256
+    assert fa.fa_bwd_workspace_size_ex(2, 3, 129, 700, 32, 1) == off + 6 * 2 * 6 * 128 * 64 * 4
+    assert fa.fa_bwd_workspace_size_ex(1, 1, 128, 0, 64, 1) == 0
+    assert fa.fa_bwd_workspace_size_ex(1, 1, 128, 128, 64, 2) == 0
+
+
 A = 0x10000  # a 16-byte aligned fake address: validation fails before any use
 
 
@@ -124,6 +137,16 @@ def test_strided_views_checked(fa_lib):
     assert fa.fa_fwd_ex(p) == -1
     assert fa_lib.fa_fwd_ex(None, None) == -1
     assert fa_lib.fa_bwd_ex(None, None) == -1
+
+
+def test_bwd_ex_deterministic_flag_checked(fa_lib):
+    t = fa.FaTensor(A, 512 * 12 * 64, 12 * 64, 64)
+    ws = fa.fa_bwd_workspace_size_ex(2, 12, 512, 512, 64, 1)
+    p = fa.BwdParams(t, t, t, t, t, A, t, t, t, 2, 12, 512, 512, 64, 0.125, 0, fa.FA_FP16, A, ws, 2)
+    assert fa.fa_bwd_ex(p) == -1                 # flag must be 0 or 1
+    p.deterministic = 1
+    p.workspace_bytes = fa.fa_bwd_workspace_size(2, 12, 512, 64)
+    assert fa.fa_bwd_ex(p) == -7                 # the plain workspace is too small for mode 1
 
 
 def test_torch_helpers_refuse_cpu_tensors(fa_lib):

@@ -103,3 +103,17 @@ def test_peak_memory_linear_in_sequence(B, H, S, D, causal):
     assert flash < 8 * io                     # O(S): outputs, gradients, workspace
     assert mat > 2 * B * H * S * S * 2        # at least two S x S fp16 tensors
     assert mat > 4 * flash
+
+
+def test_flash_attn_func_deterministic():
+    c = random_case(1, 2, 300, 300, 128, torch.bfloat16, 91)
+    grads = []
+    for _ in range(2):
+        q, k, v = (c[n].cuda().requires_grad_() for n in ("q", "k", "v"))
+        flash_attn_func(q, k, v, causal=True, deterministic=True).backward(c["do"].cuda())
+        grads.append((q.grad, k.grad, v.grad))
+    for a, b in zip(*grads):
+        assert torch.equal(a, b)
+    dq_r, _, _, _ = oracle.attention_backward(np64(c["q"]), np64(c["k"]), np64(c["v"]), np64(c["do"]),
+                                              128 ** -0.5, True)
+    check_grad(np64(grads[0][0]), dq_r, "dq")

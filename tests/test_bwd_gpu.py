@@ -106,3 +106,68 @@ def test_bwd_workloads_sampled(name):
             check_grad(dk[0, :, h], hd["dk"], f"{name} dk h{h} causal={causal}")
             check_grad(dv[0, :, h], hd["dv"], f"{name} dv h{h} causal={causal}")
             del hd
+
+
+# ----------------------------------------------------------- deterministic mode
+def _det_case(c, causal, scale=None, what=""):
+    q, k, v, do = (c[n].cuda() for n in ("q", "k", "v", "do"))
+    D = q.shape[3]
+    sc = D ** -0.5 if scale is None else scale
+    o, lse = run_fwd(q, k, v, causal, sc)
+    dq1, dk1, dv1 = fa.backward(q, k, v, o, lse, do, causal=causal, scale=sc, deterministic=True)
+    dq2, dk2, dv2 = fa.backward(q, k, v, o, lse, do, causal=causal, scale=sc, deterministic=True)
+    torch.cuda.synchronize()
+    st, detail = fa.fa_last_device_status()
+    assert st == 0, f"device status {st} {detail}"
+    for x, y, name in ((dq1, dq2, "dq"), (dk1, dk2, "dk"), (dv1, dv2, "dv")):
+        assert torch.equal(x, y), f"{what}: {name} differs between two deterministic runs"
+    qn, kn, vn, don = (np64(c[n]) for n in ("q", "k", "v", "do"))
+    dq_r, dk_r, dv_r, _ = oracle.attention_backward(qn, kn, vn, don, sc, causal)
+    for name, g, r in (("dq", dq1, dq_r), ("dk", dk1, dk_r), ("dv", dv1, dv_r)):
+        check_grad(np64(g), r, f"{what} det {name}")
+    # the atomic path sums the same fp32 blocks in another order
+    dqa, dka, dva = run_bwd(q, k, v, o, lse, do, causal, sc)
+    assert torch.equal(dka, dk1) and torch.equal(dva, dv1)
+    assert rel_l2(np64(dqa), np64(dq1)) < 2e-3
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("S", [1, 127, 129, 640])
+def test_bwd_deterministic_square(D, causal, S):
+    _det_case(random_case(1, 2, S, S, D, torch.bfloat16, 4000 + S), causal, what=f"S{S} D{D} c{causal}")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("Sq,Sk", [(100, 37), (129, 700), (700, 129), (513, 255)])
+def test_bwd_deterministic_rectangular(causal, Sq, Sk):
+    _det_case(random_case(2, 3, Sq, Sk, 128, torch.float16, 77 + Sq + Sk), causal, what=f"Sq{Sq} Sk{Sk}")
+
+
+@pytest.mark.parametrize("D", [40, 96])
+def test_bwd_deterministic_other_head_dims(D):
+    _det_case(random_case(2, 2, 300, 257, D, torch.bfloat16, 500 + D), True, what=f"D{D}")
+
+
+def test_bwd_deterministic_c4_full_size():
+    """c4 at full size in deterministic mode: two runs bit-identical, dq close
+    to the atomic path's and to the oracle on sampled rows."""
+    w = WORKLOADS["c4"]
+    inp = make_inputs(w)
+    q, k, v, do = (inp[n].cuda() for n in ("q", "k", "v", "do"))
+    o, lse = run_fwd(q, k, v, True, w.scale)
+    ws = fa.workspace_for(w.B, w.H, w.S, w.D, q.device, deterministic=True)
+    dq1, dk1, dv1 = fa.backward(q, k, v, o, lse, do, causal=True, scale=w.scale, workspace=ws, deterministic=True)
+    dq1 = dq1.clone()
+    dq2, _, _ = fa.backward(q, k, v, o, lse, do, causal=True, scale=w.scale, workspace=ws, deterministic=True)
+    torch.cuda.synchronize()
+    assert fa.fa_last_device_status()[0] == 0
+    assert torch.equal(dq1, dq2)
+    dqa, dka, dva = run_bwd(q, k, v, o, lse, do, True, w.scale)
+    assert torch.equal(dka, dk1) and torch.equal(dva, dv1)
+    assert rel_l2(np64(dqa), np64(dq1)) < 2e-3
+    rows = sample_rows(w.S, 128, 40, w.seed)
+    qn, kn, vn, don = (np64(inp[n]) for n in ("q", "k", "v", "do"))
+    got = np.stack([np64(dq1)[0, rows, h] for h in (0, w.H - 1)])
+    ref = np.stack([oracle.attention_backward_dq_rows(qn, kn, vn, don, w.scale, True, 0, h, rows) for h in (0, w.H - 1)])
+    check_grad(got, ref, "c4 det dq rows")
