@@ -170,7 +170,11 @@ struct BwdLayout {
   static constexpr int kThreads = 448;   // 14 warps
   static constexpr int BN = 128;         // keys per CTA
   static constexpr int BM = 128;         // query rows per block
-  static constexpr int QS = 2;           // Q/dO stages
+  // Q (with lse2) and dO (with Dvec) travel on separate rings: S^T(i+1)
+  // needs Q(i+1) right after dV(i), dP^T(i+1) needs dO(i+1) an iteration
+  // step later, so Q gets the deeper ring.
+  static constexpr int QS = 3;           // Q stages
+  static constexpr int OS = 1;           // dO stages
   // D = 128: dQ is computed transposed (TMEM lane = head_dim index), so each
   // warp's reductions into the accumulator cover one contiguous 128-byte line.
   static constexpr bool DQ_T = (D == 128);
@@ -182,13 +186,13 @@ struct BwdLayout {
   static constexpr int OFF_V = OFF_K + TILE;
   static constexpr int OFF_Q = OFF_V + TILE;
   static constexpr int OFF_DO = OFF_Q + QS * TILE;
-  static constexpr int OFF_DS = OFF_DO + QS * TILE;
+  static constexpr int OFF_DS = OFF_DO + OS * TILE;
   static constexpr int OFF_LSE = OFF_DS + DS_TILE;
   static constexpr int OFF_DVEC = OFF_LSE + QS * BM * 4;
-  static constexpr int OFF_BAR = OFF_DVEC + QS * BM * 4;
-  // kv_full, q_full[QS], q_empty[QS], sx_full, dp_full, p_ready, ds_ready,
-  // ds_free, dq_full, dq_free, mma_done, drain
-  static constexpr int NBAR = 1 + 2 * QS + 10;
+  static constexpr int OFF_BAR = OFF_DVEC + OS * BM * 4;
+  // kv_full, q_full[QS], q_empty[QS], o_full[OS], o_empty[OS], sx_full,
+  // dp_full, p_ready, ds_ready, ds_free, dq_full, dq_free, mma_done, drain
+  static constexpr int NBAR = 1 + 2 * QS + 2 * OS + 9;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int SMEM_MAX = 232448;
@@ -231,7 +235,9 @@ __global__ void __launch_bounds__(448, 1)
   uint64_t* kv_full = bars;
   uint64_t* q_full = kv_full + 1;
   uint64_t* q_empty = q_full + QS;
-  uint64_t* sx_full = q_empty + QS;
+  uint64_t* o_full = q_empty + QS;
+  uint64_t* o_empty = o_full + L::OS;
+  uint64_t* sx_full = o_empty + L::OS;
   uint64_t* dp_full = sx_full + 1;
   uint64_t* p_ready = dp_full + 1;
   uint64_t* ds_ready = p_ready + 1;
@@ -263,6 +269,10 @@ __global__ void __launch_bounds__(448, 1)
     for (int s = 0; s < QS; ++s) {
       mbar_init(&q_full[s], 1);
       mbar_init(&q_empty[s], 1);
+    }
+    for (int s = 0; s < L::OS; ++s) {
+      mbar_init(&o_full[s], 1);
+      mbar_init(&o_empty[s], 1);
     }
     mbar_init(sx_full, 1);
     mbar_init(dp_full, 1);
@@ -300,23 +310,41 @@ __global__ void __launch_bounds__(448, 1)
           tma_load_4d(smem + L::OFF_K + kb * L::BLK, &tmK, kv_full, kb * 64, n0, h, b);
           tma_load_4d(smem + L::OFF_V + kb * L::BLK, &tmV, kv_full, kb * 64, n0, h, b);
         }
-        int i = 0;
-        for (; i < n; ++i) {
-          const int st = i % QS;
-          const uint32_t ph = (i / QS) & 1;
-          if (!wait_bar(&q_empty[st], ph ^ 1, abort_flag, kRoleLoader, i)) break;
-          const int i0 = (i_start + i) * BM;
-          mbar_arrive_expect_tx(&q_full[st], 2 * L::TILE + 2 * BM * 4);
-          for (int kb = 0; kb < L::KB; ++kb) {
-            tma_load_4d(smem + L::OFF_Q + st * L::TILE + kb * L::BLK, &tmQ, &q_full[st], kb * 64, i0, h, b);
-            tma_load_4d(smem + L::OFF_DO + st * L::TILE + kb * L::BLK, &tmdO, &q_full[st], kb * 64, i0, h, b);
-          }
-          bulk_load(smem + L::OFF_LSE + st * BM * 4, a.lse2 + bh_row0 + i0, BM * 4, &q_full[st]);
-          bulk_load(smem + L::OFF_DVEC + st * BM * 4, a.dvec + bh_row0 + i0, BM * 4, &q_full[st]);
+        // Q(j) with lse2(j) runs QS - 1 blocks ahead of dO(j) with Dvec(j):
+        // per step, dO(i) (its slot frees first) and then Q(i + QS - 1).
+        int nq = 0, no = 0;  // loads issued
+        auto load_q = [&](int j) -> bool {
+          const int st = j % QS;
+          if (!wait_bar(&q_empty[st], ((j / QS) & 1) ^ 1, abort_flag, kRoleLoader, j)) return false;
+          const int j0 = (i_start + j) * BM;
+          mbar_arrive_expect_tx(&q_full[st], L::TILE + BM * 4);
+          for (int kb = 0; kb < L::KB; ++kb)
+            tma_load_4d(smem + L::OFF_Q + st * L::TILE + kb * L::BLK, &tmQ, &q_full[st], kb * 64, j0, h, b);
+          bulk_load(smem + L::OFF_LSE + st * BM * 4, a.lse2 + bh_row0 + j0, BM * 4, &q_full[st]);
+          ++nq;
+          return true;
+        };
+        auto load_o = [&](int j) -> bool {
+          const int st = j % L::OS;
+          if (!wait_bar(&o_empty[st], ((j / L::OS) & 1) ^ 1, abort_flag, kRoleLoader, j)) return false;
+          const int j0 = (i_start + j) * BM;
+          mbar_arrive_expect_tx(&o_full[st], L::TILE + BM * 4);
+          for (int kb = 0; kb < L::KB; ++kb)
+            tma_load_4d(smem + L::OFF_DO + st * L::TILE + kb * L::BLK, &tmdO, &o_full[st], kb * 64, j0, h, b);
+          bulk_load(smem + L::OFF_DVEC + st * BM * 4, a.dvec + bh_row0 + j0, BM * 4, &o_full[st]);
+          ++no;
+          return true;
+        };
+        bool lok = true;
+        for (int j = 0; lok && j < QS - 1 && j < n; ++j) lok = load_q(j);
+        for (int i = 0; lok && i < n; ++i) {
+          lok = load_o(i);
+          if (lok && i + QS - 1 < n) lok = load_q(i + QS - 1);
         }
         if (*abort_flag) {
           drain_wait(kv_full, 0);
-          for (int j = max(0, i - QS); j < i; ++j) drain_wait(&q_full[j % QS], (j / QS) & 1);
+          for (int j = max(0, nq - QS); j < nq; ++j) drain_wait(&q_full[j % QS], (j / QS) & 1);
+          for (int j = max(0, no - L::OS); j < no; ++j) drain_wait(&o_full[j % L::OS], (j / L::OS) & 1);
         }
       }
     } else if (warp == kMmaWarp) {
@@ -347,14 +375,19 @@ __global__ void __launch_bounds__(448, 1)
           tc_fence_after();
           issue_kt(L::COL_X, sK, sQ);
           mma_commit(sx_full);
+          ok = wait_bar(&o_full[0], 0, abort_flag, kRoleMma, 0);
+        }
+        if (ok) {
+          tc_fence_after();
           issue_kt(L::COL_Y, sV, sdO);
           mma_commit(dp_full);
         }
         for (int i = 0; ok && i < n; ++i) {
           const int st = i % QS;
           const uint32_t ph = i & 1;
+          const int ost = i % L::OS;
           const uint32_t qa = sQ + st * L::TILE;
-          const uint32_t da = sdO + st * L::TILE;
+          const uint32_t da = sdO + ost * L::TILE;
           if (!(ok = wait_bar(p_ready, ph, abort_flag, kRoleMma, i))) break;
           tc_fence_after();
           // dV += P^T dO
@@ -374,6 +407,9 @@ __global__ void __launch_bounds__(448, 1)
           }
           if (!(ok = wait_bar(ds_ready, ph, abort_flag, kRoleMma, i))) break;
           tc_fence_after();
+          // dO(i) and Dvec(i) are free once dV(i) is done (the softmax warps
+          // have read Dvec(i): ds_ready).
+          mma_commit(&o_empty[ost]);
           // dQ (or dQ^T) into Y first, so that its drain overlaps dK(i): dP^T(i)
           // there has been read by the softmax warps.
 #pragma unroll
@@ -397,10 +433,11 @@ __global__ void __launch_bounds__(448, 1)
           mma_commit(ds_free);
           if (i + 1 < n) {
             // dP^T(i+1) into Y once dQ(i) has been read out of it.
-            const int sn = (i + 1) % QS;
+            const int on = (i + 1) % L::OS;
             if (!(ok = wait_bar(dq_free, ph, abort_flag, kRoleMma, i))) break;
+            if (!(ok = wait_bar(&o_full[on], ((i + 1) / L::OS) & 1, abort_flag, kRoleMma, i + 1))) break;
             tc_fence_after();
-            issue_kt(L::COL_Y, sV, sdO + sn * L::TILE);
+            issue_kt(L::COL_Y, sV, sdO + on * L::TILE);
             mma_commit(dp_full);
           }
         }
@@ -431,7 +468,7 @@ __global__ void __launch_bounds__(448, 1)
       int cmin = a.causal ? key - off - i0 : -1;
       if (key >= a.Sk) cmin = BM;
       const float* lse_s = s_lse + st * BM + 64 * g;
-      const float* dvec_s = s_dvec + st * BM + 64 * g;
+      const float* dvec_s = s_dvec + (i % L::OS) * BM + 64 * g;
       const int cm = cmin - 64 * g;  // in this warpgroup's column numbering
       // Phase A: P^T = 2^(S^T scale log2e - lse2) -> 16-bit pairs into X.
       uint32_t pp[2][16];
@@ -491,7 +528,8 @@ __global__ void __launch_bounds__(448, 1)
       // Phase B: dS^T = P^T (dP^T - Dvec) -> 16-bit pairs into swizzled smem
       // (the A operand of dK, the B operand of dQ^T / A of dQ).
       ok = __all_sync(0xffffffffu, wait_bar(dp_full, ph, abort_flag, kRoleSoftmax, i) &&
-                                       wait_bar(ds_free, ph ^ 1, abort_flag, kRoleSoftmax, i));
+                                       wait_bar(ds_free, ph ^ 1, abort_flag, kRoleSoftmax, i) &&
+                                       wait_bar(&o_full[i % L::OS], (i / L::OS) & 1, abort_flag, kRoleSoftmax, i));
       if (!ok) break;
       tc_fence_after();
       const uint32_t ds_row = smem_u32(smem + L::OFF_DS + g * L::BLK) + kr * 128;
