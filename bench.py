@@ -288,9 +288,35 @@ def run_ours(args, w, causal):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
+        t_seq = max_over_ranks(e0.elapsed_time(e1) / 1e3, dev)
+
+        # The public host-memory API: HostAttentionPipeline overlaps step k's
+        # kernels with step k+1's inputs arriving and step k-1's results
+        # leaving (three streams, two device buffer sets). Every step still
+        # copies all its inputs in and all its results out.
+        from exact_io_aware_96_b200.host_pipeline import HostAttentionPipeline
+        pipe = HostAttentionPipeline(B, S, H, D, dtype=q.dtype, causal=causal, scale=w.scale, device=dev)
+        for _ in range(max(2, args.warmup)):
+            pipe.step(hq, hk, hv, hdo, ho, hl, hdq, hdk, hdv)
+        pipe.synchronize()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0.record(stream)
+        pipe.start_after(stream)
+        for _ in range(n_e2e):
+            pipe.step(hq, hk, hv, hdo, ho, hl, hdq, hdk, hdv)
+        pipe.join(stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
         t_e2e = max_over_ranks(e0.elapsed_time(e1) / 1e3, dev)
         e2e = {"value": (ff + fb) * n_e2e * world / t_e2e / 1e12, "unit": "TFLOP/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e,
+               "api": "exact_io_aware_96_b200.host_pipeline.HostAttentionPipeline (pinned host buffers; "
+                      "copies overlapped with neighbouring steps' kernels)",
+               "sequential_value": (ff + fb) * n_e2e * world / t_seq / 1e12,
+               "sequential_api": "copy in, fa.forward + fa.backward, copy out, one step after another"}
+        del pipe
 
     peaks, peaks_src = load_peaks()
     timed_s = t_fwd + t_bwd

@@ -470,6 +470,12 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, c
   return fa_bwd_ex(&p, stream);
 }
 
+int fa_selftest_wait_timeout(unsigned int limit_us, fa_stream_t stream) {
+  if (limit_us < 1 || limit_us > 4000000u) return FA_ERR_INVALID_ARG;
+  fa::fa_selftest_wait_kernel<<<1, 64, 0, reinterpret_cast<cudaStream_t>(stream)>>>(uint64_t(limit_us) * 1000u);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 int fa_last_device_status(int* detail) {
   if (cudaDeviceSynchronize() != cudaSuccess) return FA_ERR_CUDA;
   int h[4] = {0, 0, 0, 0};

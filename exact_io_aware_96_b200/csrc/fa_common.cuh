@@ -17,7 +17,7 @@ namespace fa {
 // its own copy of a __device__ variable).
 __device__ int g_status[4];
 
-enum Role : int { kRoleLoader = 1, kRoleMma = 2, kRoleSoftmax = 3 };
+enum Role : int { kRoleLoader = 1, kRoleMma = 2, kRoleSoftmax = 3, kRoleSelfTest = 4 };
 
 // A wait longer than this is treated as a hang: the kernel records it and
 // winds down instead of spinning forever. Real waits last microseconds.
@@ -35,13 +35,13 @@ __device__ __forceinline__ void record_timeout(int role, int iter) {
 // CTA-wide abort flag) if it has not after kWaitLimitNs, or if another warp of
 // the CTA has already aborted.
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int role,
-                                         int iter) {
+                                         int iter, uint64_t limit_ns = kWaitLimitNs) {
   if (sm100::mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = sm100::globaltimer_ns();
   while (true) {
     if (sm100::mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (sm100::globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (sm100::globaltimer_ns() - t0 > limit_ns) {
       *abort_flag = 1;
       record_timeout(role, iter);
       return false;
@@ -56,6 +56,27 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   while (!sm100::mbar_try_wait(bar, parity)) {
     if (sm100::globaltimer_ns() - t0 > 500000000ull) break;
   }
+}
+
+// Self-test of the failure path: warp 0 waits on an mbarrier that nothing
+// arrives on, with a limit of limit_ns; it records the timeout in the status
+// word and raises the block's abort flag. Warp 1 waits on the same barrier
+// with the normal limit and leaves as soon as it sees the abort flag, the way
+// the other roles of a pipeline wind down.
+__global__ void __launch_bounds__(64) fa_selftest_wait_kernel(uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(&bar, 1);
+    abort_flag = 0;
+    sm100::fence_mbar_init();
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5;
+  if (warp == 0)
+    wait_bar(&bar, 0, &abort_flag, kRoleSelfTest, 0, limit_ns);
+  else
+    wait_bar(&bar, 0, &abort_flag, kRoleSelfTest, 1);
 }
 
 struct FwdArgs {

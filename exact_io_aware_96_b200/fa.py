@@ -24,7 +24,8 @@ STATUS = {
 }
 FA_NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 EXPORTED = ("fa_fwd", "fa_fwd_ex", "fa_fwd_fp8", "fa_fwd_fp8_ex", "fa_bwd", "fa_bwd_ex", "fa_bwd_noalloc",
-            "fa_bwd_workspace_size", "fa_bwd_workspace_size_ex", "fa_last_device_status", "fa_strerror", "fa_version")
+            "fa_bwd_workspace_size", "fa_bwd_workspace_size_ex", "fa_selftest_wait_timeout",
+            "fa_last_device_status", "fa_strerror", "fa_version")
 
 
 class FaTensor(ctypes.Structure):
@@ -94,6 +95,8 @@ def lib():
         L.fa_bwd_workspace_size.restype = sz
         L.fa_bwd_workspace_size_ex.argtypes = [i, i, i, i, i, i]
         L.fa_bwd_workspace_size_ex.restype = sz
+        L.fa_selftest_wait_timeout.argtypes = [ctypes.c_uint, vp]
+        L.fa_selftest_wait_timeout.restype = i
         L.fa_last_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
         L.fa_last_device_status.restype = i
         L.fa_strerror.argtypes = [i]
@@ -145,6 +148,11 @@ def fa_bwd_workspace_size(B, H, Sq, D) -> int:
 
 def fa_bwd_workspace_size_ex(B, H, Sq, Sk, D, deterministic) -> int:
     return lib().fa_bwd_workspace_size_ex(B, H, Sq, Sk, D, deterministic)
+
+
+def fa_selftest_wait_timeout(limit_us, stream=0) -> int:
+    """Launch the failure-path self-test (see include/fa.h)."""
+    return lib().fa_selftest_wait_timeout(limit_us, stream)
 
 
 def fa_last_device_status():

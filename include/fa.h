@@ -249,8 +249,17 @@ size_t fa_bwd_workspace_size_ex(int B, int H, int Sq, int Sk, int D, int determi
    kernels since the last call (FA_OK or FA_ERR_TIMEOUT) and clears it.
    FA_ERR_CUDA if the device cannot be queried. If `detail` is non-null it
    receives 4 ints: code, linear block index, role (1 = loader, 2 = MMA
-   issuer, 3 = softmax/epilogue) and the block-loop iteration. */
+   issuer, 3 = softmax/epilogue, 4 = self-test) and the block-loop iteration. */
 int fa_last_device_status(int* detail);
+
+/* Self-test of failure detection (not a method step). Launches one block on
+   `stream` whose pipeline wait never completes: after limit_us microseconds
+   (1 .. 4,000,000) the wait gives up, records FA_ERR_TIMEOUT in the device
+   status word with role 4 (self-test) and block 0, and the block winds down
+   through the same abort path the attention kernels use. Nothing faults or
+   hangs and the context stays usable; read the result with
+   fa_last_device_status(). FA_ERR_INVALID_ARG for a limit out of range. */
+int fa_selftest_wait_timeout(unsigned int limit_us, fa_stream_t stream);
 
 /* Static, human-readable text for a status code. Never null. */
 const char* fa_strerror(int status);

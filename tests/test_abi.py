@@ -149,6 +149,11 @@ def test_bwd_ex_deterministic_flag_checked(fa_lib):
     assert fa.fa_bwd_ex(p) == -7                 # the plain workspace is too small for mode 1
 
 
+def test_selftest_limit_checked(fa_lib):
+    assert fa.fa_selftest_wait_timeout(0) == -1
+    assert fa.fa_selftest_wait_timeout(4000001) == -1
+
+
 def test_torch_helpers_refuse_cpu_tensors(fa_lib):
     import torch
     q = torch.zeros(1, 8, 1, 64, dtype=torch.float16)
@@ -156,3 +161,12 @@ def test_torch_helpers_refuse_cpu_tensors(fa_lib):
         fa.forward(q, q, q)
     with pytest.raises(TypeError):
         fa.forward(q.float(), q.float(), q.float())
+
+
+def test_host_pipeline_needs_a_gpu():
+    import torch
+    from exact_io_aware_96_b200.host_pipeline import HostAttentionPipeline
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    with pytest.raises(RuntimeError):
+        HostAttentionPipeline(1, 128, 2, 64)
