@@ -27,9 +27,14 @@
 //               columns [0, 64), warps 4-7 [64, 128). At the end warps 0-3
 //               write dK and warps 4-7 write dV.
 //   warps 8-11  read the dQ block out of TMEM and add it into the fp32
-//               accumulator (D = 128: dQ^T, one head_dim index per thread, so
-//               a warp's reductions hit one 128-byte line per query)
-//   warp  12    TMA loader: K, V once; Q_i, dO_i, lse2_i, Dvec_i per query block
+//               accumulator. D = 128: dQ^T (one head_dim index per thread),
+//               staged in shared memory a quarter (32 query rows) at a time
+//               and added by TMA bulk reductions, which keeps the reduction
+//               traffic off the load/store queues the softmax warps use.
+//               D = 64: red.global.add.v4 per query row. Deterministic mode:
+//               plain stores into the block's own slot.
+//   warp  12    TMA loader: K, V once; Q_i with lse2_i and dO_i with Dvec_i per
+//               query block, on separate rings (Q runs ahead of dO)
 //   warp  13    MMA issuer
 // Blocks are 128 keys x 128 queries. Tensor memory: dK and dV accumulators,
 // X (S^T, then 16-bit P^T written back by the softmax warps and used as the
@@ -171,9 +176,11 @@ struct BwdLayout {
   static constexpr int BN = 128;         // keys per CTA
   static constexpr int BM = 128;         // query rows per block
   // Q (with lse2) and dO (with Dvec) travel on separate rings: S^T(i+1)
-  // needs Q(i+1) right after dV(i), dP^T(i+1) needs dO(i+1) an iteration
-  // step later, so Q gets the deeper ring.
-  static constexpr int QS = 3;           // Q stages
+  // needs Q(i+1) right after dV(i), dP^T(i+1) needs dO(i+1) later in block
+  // i, after dO(i) has been released, so one dO stage suffices.
+  // Q stages: three where shared memory allows (D = 64); D = 128 spends the
+  // third stage's 32 KB on the dQ staging buffers below.
+  static constexpr int QS = (D == 128) ? 2 : 3;
   static constexpr int OS = 1;           // dO stages
   // D = 128: dQ is computed transposed (TMEM lane = head_dim index), so each
   // warp's reductions into the accumulator cover one contiguous 128-byte line.
@@ -187,7 +194,11 @@ struct BwdLayout {
   static constexpr int OFF_Q = OFF_V + TILE;
   static constexpr int OFF_DO = OFF_Q + QS * TILE;
   static constexpr int OFF_DS = OFF_DO + OS * TILE;
-  static constexpr int OFF_LSE = OFF_DS + DS_TILE;
+  // D = 128: two 16 KB staging buffers, each 32 query rows x 128 fp32 of a
+  // dQ block, from which the TMA adds the block into the accumulator.
+  static constexpr int DQ_PART = 32 * 128 * 4;
+  static constexpr int OFF_DQS = OFF_DS + DS_TILE;
+  static constexpr int OFF_LSE = OFF_DQS + (DQ_T ? 2 * DQ_PART : 0);
   static constexpr int OFF_DVEC = OFF_LSE + QS * BM * 4;
   static constexpr int OFF_BAR = OFF_DVEC + OS * BM * 4;
   // kv_full, q_full[QS], q_empty[QS], o_full[OS], o_empty[OS], sx_full,
@@ -616,7 +627,10 @@ __global__ void __launch_bounds__(448, 1)
           red_add_f32(p, x);
       };
       for (int i = 0; i < n; ++i) {
-        const bool ok = __all_sync(0xffffffffu, wait_bar(dq_full, i & 1, abort_flag, kRoleSoftmax, i));
+        bool ok = __all_sync(0xffffffffu, wait_bar(dq_full, i & 1, abort_flag, kRoleSoftmax, i));
+        // The staged path synchronises the four drain warps on a named
+        // barrier, so they must all go on or all stop.
+        if constexpr (L::DQ_T && !DET) ok = named_bar_and(1, 128, ok);
         if (!ok) break;
         tc_fence_after();
         const int qb = i_start + i;
@@ -636,17 +650,50 @@ __global__ void __launch_bounds__(448, 1)
           tmem_ld_wait();
 #pragma unroll
           for (int part = 0; part < 3; ++part) reg_fence(v[part]);
+          if constexpr (DET) {
 #pragma unroll
-          for (int c = 0; c < 32; ++c) put(col + c * D, __uint_as_float(v[0][c]));
-          tmem_ld32(tY + 96, v[0]);
-          tmem_ld_wait();
-          reg_fence(v[0]);
-          tc_fence_before();
-          mbar_arrive(dq_free);  // Y may take dP^T(i+1) now
+            for (int c = 0; c < 32; ++c) put(col + c * D, __uint_as_float(v[0][c]));
+            tmem_ld32(tY + 96, v[0]);
+            tmem_ld_wait();
+            reg_fence(v[0]);
+            tc_fence_before();
+            mbar_arrive(dq_free);  // Y may take dP^T(i+1) now
 #pragma unroll
-          for (int part = 1; part < 4; ++part)
+            for (int part = 1; part < 4; ++part)
 #pragma unroll
-            for (int c = 0; c < 32; ++c) put(col + (32 * part + c) * D, __uint_as_float(v[part == 3 ? 0 : part][c]));
+              for (int c = 0; c < 32; ++c)
+                put(col + (32 * part + c) * D, __uint_as_float(v[part == 3 ? 0 : part][c]));
+          } else {
+            // Quarter p (32 query rows) goes to staging buffer p & 1 as rows of
+            // 128 floats (each warp writes 128 contiguous bytes per row), then
+            // one thread has the TMA add the 16 KB into the accumulator, where
+            // the same 32 rows are contiguous. A buffer is rewritten only after
+            // the TMA has finished reading it.
+            const uint32_t stage0 = smem_u32(smem + L::OFF_DQS);
+            auto stage = [&](int part, const uint32_t (&x)[32]) {
+              const uint32_t buf = stage0 + (part & 1) * L::DQ_PART;
+              if (warp == 8 && lane == 0) bulk_wait_read1();  // the group that read this buffer last
+              __syncwarp();
+              named_bar_sync(1, 128);
+#pragma unroll
+              for (int c = 0; c < 32; ++c) st_shared_f32(buf + (c * D + tr) * 4, __uint_as_float(x[c]));
+              fence_proxy_async_smem();
+              named_bar_sync(1, 128);
+              if (warp == 8 && lane == 0) {
+                bulk_reduce_add_f32(base + 32 * part * D, smem + L::OFF_DQS + (part & 1) * L::DQ_PART, L::DQ_PART);
+                bulk_commit();
+              }
+            };
+            stage(0, v[0]);
+            tmem_ld32(tY + 96, v[0]);
+            tmem_ld_wait();
+            reg_fence(v[0]);
+            tc_fence_before();
+            mbar_arrive(dq_free);  // Y may take dP^T(i+1) now
+            stage(1, v[1]);
+            stage(2, v[2]);
+            stage(3, v[0]);
+          }
         } else {
           // lane = query row, columns = head_dim (64): the whole block fits in
           // registers, so Y is released before the writes.
@@ -673,10 +720,13 @@ __global__ void __launch_bounds__(448, 1)
         }
       }
     };
-    if (a.dq_part != nullptr)
+    if (a.dq_part != nullptr) {
       drain(std::true_type{});
-    else
+    } else {
       drain(std::false_type{});
+      // Let the TMA finish the last reductions before shared memory goes away.
+      if (L::DQ_T && warp == 8 && lane == 0) bulk_wait0();
+    }
   }
 
   tc_fence_before();
