@@ -374,13 +374,18 @@ __global__ void __launch_bounds__(448, 1)
         // MN-major, B = dS^T MN-major. D = 64: dQ = dS K, M = 128 queries, N = D; A = dS^T
         // viewed MN-major, B = K MN-major.
         const uint32_t id_q = L::DQ_T ? idesc_f16(BF16, 128, 128, 1, 1) : idesc_f16(BF16, 128, D, 1, 1);
+        // Operand descriptors are formed once per tile and advanced by adds.
         auto issue_kt = [&](uint32_t dcol, uint32_t kv, uint32_t qa) {  // dcol = kv-tile x qa-tile^T
+          const uint64_t a0 = desc_sw128(kv, 16, 1024), b0 = desc_sw128(qa, 16, 1024);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t o = (kk >> 2) * L::BLK + (kk & 3) * 32;
-            mma_ss(tmem + dcol, desc_sw128(kv + o, 16, 1024), desc_sw128(qa + o, 16, 1024), id_s, kk > 0);
+            mma_ss(tmem + dcol, desc_add(a0, o), desc_add(b0, o), id_s, kk > 0);
           }
         };
+        const uint64_t ds_k = desc_sw128(sDS, 16, 1024);         // dS^T, K-major (A of dK)
+        const uint64_t ds_mn = desc_sw128(sDS, L::BLK, 1024);    // dS^T, MN-major (dQ)
+        const uint64_t k_mn = desc_sw128(sK, L::BLK, 1024);      // K, MN-major (dQ)
         bool ok = wait_bar(kv_full, 0, abort_flag, kRoleMma, -1) && wait_bar(&q_full[0], 0, abort_flag, kRoleMma, 0);
         if (ok) {
           tc_fence_after();
@@ -398,13 +403,14 @@ __global__ void __launch_bounds__(448, 1)
           const uint32_t ph = i & 1;
           const int ost = i % L::OS;
           const uint32_t qa = sQ + st * L::TILE;
-          const uint32_t da = sdO + ost * L::TILE;
+          const uint64_t q_mn = desc_sw128(qa, L::BLK, 1024);
+          const uint64_t do_mn = desc_sw128(sdO + ost * L::TILE, L::BLK, 1024);
           if (!(ok = wait_bar(p_ready, ph, abort_flag, kRoleMma, i))) break;
           tc_fence_after();
           // dV += P^T dO
 #pragma unroll
           for (int kk = 0; kk < BM / 16; ++kk)
-            mma_ts(tmem + L::COL_DV, tmem + L::col_p(kk), desc_sw128(da + kk * 2048, L::BLK, 1024), id_kv,
+            mma_ts(tmem + L::COL_DV, tmem + L::col_p(kk), desc_add(do_mn, kk * 2048), id_kv,
                    (i > 0 || kk > 0) ? 1u : 0u);
           if (i + 1 < n) {
             // S^T(i+1) into X as soon as dV(i) has been issued: X held only
@@ -425,8 +431,8 @@ __global__ void __launch_bounds__(448, 1)
           // there has been read by the softmax warps.
 #pragma unroll
           for (int kk = 0; kk < L::BN / 16; ++kk) {
-            const uint64_t dk_desc = desc_sw128(sDS + kk * 2048, L::BLK, 1024);
-            const uint64_t k_desc = desc_sw128(sK + kk * 2048, L::BLK, 1024);
+            const uint64_t dk_desc = desc_add(ds_mn, kk * 2048);
+            const uint64_t k_desc = desc_add(k_mn, kk * 2048);
             if constexpr (L::DQ_T)
               mma_ss(tmem + L::COL_Y, k_desc, dk_desc, id_q, kk > 0);
             else
@@ -437,7 +443,7 @@ __global__ void __launch_bounds__(448, 1)
 #pragma unroll
           for (int kk = 0; kk < BM / 16; ++kk) {
             const uint32_t o = (kk >> 2) * L::BLK + (kk & 3) * 32;
-            mma_ss(tmem + L::COL_DK, desc_sw128(sDS + o, 16, 1024), desc_sw128(qa + kk * 2048, L::BLK, 1024), id_kv,
+            mma_ss(tmem + L::COL_DK, desc_add(ds_k, o), desc_add(q_mn, kk * 2048), id_kv,
                    (i > 0 || kk > 0) ? 1u : 0u);
           }
           mma_commit(&q_empty[st]);
@@ -670,7 +676,7 @@ __global__ void __launch_bounds__(448, 1)
             // the same 32 rows are contiguous. A buffer is rewritten only after
             // the TMA has finished reading it.
             const uint32_t stage0 = smem_u32(smem + L::OFF_DQS);
-            auto stage = [&](int part, const uint32_t (&x)[32]) {
+            auto store = [&](int part, const uint32_t (&x)[32]) {
               const uint32_t buf = stage0 + (part & 1) * L::DQ_PART;
               if (warp == 8 && lane == 0) bulk_wait_read1();  // the group that read this buffer last
               __syncwarp();
@@ -678,21 +684,27 @@ __global__ void __launch_bounds__(448, 1)
 #pragma unroll
               for (int c = 0; c < 32; ++c) st_shared_f32(buf + (c * D + tr) * 4, __uint_as_float(x[c]));
               fence_proxy_async_smem();
+            };
+            auto reduce = [&](int part) {
               named_bar_sync(1, 128);
               if (warp == 8 && lane == 0) {
                 bulk_reduce_add_f32(base + 32 * part * D, smem + L::OFF_DQS + (part & 1) * L::DQ_PART, L::DQ_PART);
                 bulk_commit();
               }
             };
-            stage(0, v[0]);
+            store(0, v[0]);
             tmem_ld32(tY + 96, v[0]);
             tmem_ld_wait();
             reg_fence(v[0]);
             tc_fence_before();
             mbar_arrive(dq_free);  // Y may take dP^T(i+1) now
-            stage(1, v[1]);
-            stage(2, v[2]);
-            stage(3, v[0]);
+            reduce(0);
+            store(1, v[1]);
+            reduce(1);
+            store(2, v[2]);
+            reduce(2);
+            store(3, v[0]);
+            reduce(3);
           }
         } else {
           // lane = query row, columns = head_dim (64): the whole block fits in

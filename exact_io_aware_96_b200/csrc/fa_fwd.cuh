@@ -188,28 +188,28 @@ __global__ void __launch_bounds__(320, 1)
       const uint32_t sK = smem_u32(smem + L::OFF_K);
       const uint32_t sV = smem_u32(smem + L::OFF_V);
       auto issue_S = [&](int t, int st) {
-        const uint32_t qa = sQ + t * L::TILE;
-        const uint32_t ka = sK + st * L::TILE;
+        const uint64_t qd = desc_sw128(sQ + t * L::TILE, 16, 1024);
+        const uint64_t kd = desc_sw128(sK + st * L::TILE, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < L::RB / 32; ++kk) {  // 32 bytes of K per instruction
           const uint32_t o = (kk >> 2) * L::BLK + (kk & 3) * 32;
           if constexpr (FP8)
-            mma_ss_f8(tmem + t * 128, desc_sw128(qa + o, 16, 1024), desc_sw128(ka + o, 16, 1024), idS, kk > 0);
+            mma_ss_f8(tmem + t * 128, desc_add(qd, o), desc_add(kd, o), idS, kk > 0);
           else
-            mma_ss(tmem + t * 128, desc_sw128(qa + o, 16, 1024), desc_sw128(ka + o, 16, 1024), idS, kk > 0);
+            mma_ss(tmem + t * 128, desc_add(qd, o), desc_add(kd, o), idS, kk > 0);
         }
       };
       auto issue_PV = [&](int t, int st, int acc) {
-        const uint32_t va = sV + st * L::TILE;
+        const uint64_t vd = desc_sw128(sV + st * L::TILE, L::BLK, 1024);
         // P occupies 8 TMEM columns per instruction (16 keys of 16-bit, 32
         // keys of e4m3); V advances by as many 128-byte rows.
 #pragma unroll
         for (int kk = 0; kk < (FP8 ? 4 : 8); ++kk) {
           if constexpr (FP8)
-            mma_ts_f8(tmem + 256 + t * D, tmem + t * 128 + kk * 8, desc_sw128(va + kk * 4096, L::BLK, 1024), idO,
+            mma_ts_f8(tmem + 256 + t * D, tmem + t * 128 + kk * 8, desc_add(vd, kk * 4096), idO,
                       (acc || kk > 0) ? 1u : 0u);
           else
-            mma_ts(tmem + 256 + t * D, tmem + t * 128 + kk * 8, desc_sw128(va + kk * 2048, L::BLK, 1024), idO,
+            mma_ts(tmem + 256 + t * D, tmem + t * 128 + kk * 8, desc_add(vd, kk * 2048), idO,
                    (acc || kk > 0) ? 1u : 0u);
         }
       };

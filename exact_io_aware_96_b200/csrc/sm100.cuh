@@ -284,6 +284,12 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t lbo, uin
   return d;
 }
 
+// The descriptor of an operand `bytes` further on in shared memory (bytes a
+// multiple of 16): the start address field holds address >> 4 in 14 bits and
+// every shared-memory address here stays below 2^18, so the add cannot carry
+// out of the field.
+__device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
+
 // Instruction descriptor of tcgen05.mma kind::f16 with fp32 accumulation.
 // is_bf16: both operands bf16 (else both fp16). a_mn / b_mn: operand stored
 // MN-major (else K-major).
