@@ -194,11 +194,12 @@ struct BwdLayout {
   static constexpr int OFF_Q = OFF_V + TILE;
   static constexpr int OFF_DO = OFF_Q + QS * TILE;
   static constexpr int OFF_DS = OFF_DO + OS * TILE;
-  // D = 128: two 16 KB staging buffers, each 32 query rows x 128 fp32 of a
-  // dQ block, from which the TMA adds the block into the accumulator.
-  static constexpr int DQ_PART = 32 * 128 * 4;
+  // dQ staging, from which the TMA adds a dQ block into the accumulator.
+  // D = 128: two 16 KB buffers, each 32 query rows x 128 fp32. D = 64: one
+  // 8 KB buffer per drain warp (its 32 query rows x 64 fp32).
+  static constexpr int DQ_PART = 32 * D * 4;
   static constexpr int OFF_DQS = OFF_DS + DS_TILE;
-  static constexpr int OFF_LSE = OFF_DQS + (DQ_T ? 2 * DQ_PART : 0);
+  static constexpr int OFF_LSE = OFF_DQS + (DQ_T ? 2 * DQ_PART : 4 * DQ_PART);
   static constexpr int OFF_DVEC = OFF_LSE + QS * BM * 4;
   static constexpr int OFF_BAR = OFF_DVEC + OS * BM * 4;
   // kv_full, q_full[QS], q_empty[QS], o_full[OS], o_empty[OS], sx_full,
@@ -718,17 +719,34 @@ __global__ void __launch_bounds__(448, 1)
           for (int part = 0; part < D / 32; ++part) reg_fence(v[part]);
           tc_fence_before();
           mbar_arrive(dq_free);
+          if constexpr (DET) {
 #pragma unroll
-          for (int part = 0; part < D / 32; ++part)
+            for (int part = 0; part < D / 32; ++part)
 #pragma unroll
-            for (int c = 0; c < 32; c += 4) {
-              const float x0 = __uint_as_float(v[part][c]), x1 = __uint_as_float(v[part][c + 1]);
-              const float x2 = __uint_as_float(v[part][c + 2]), x3 = __uint_as_float(v[part][c + 3]);
-              if constexpr (DET)
-                *reinterpret_cast<float4*>(row + 32 * part + c) = make_float4(x0, x1, x2, x3);
-              else
-                red_add_v4_f32(row + 32 * part + c, x0, x1, x2, x3);
+              for (int c = 0; c < 32; c += 4)
+                *reinterpret_cast<float4*>(row + 32 * part + c) =
+                    make_float4(__uint_as_float(v[part][c]), __uint_as_float(v[part][c + 1]),
+                                __uint_as_float(v[part][c + 2]), __uint_as_float(v[part][c + 3]));
+          } else {
+            // This warp's 32 rows are contiguous in the accumulator: stage
+            // them as rows of D floats and let the TMA add the 8 KB.
+            const int wq = warp & 3;
+            uint8_t* wbuf = smem + L::OFF_DQS + wq * L::DQ_PART;
+            if (lane == 0) bulk_wait_read0();  // this warp's previous reduction has read the buffer
+            __syncwarp();
+            const uint32_t rbuf = smem_u32(wbuf) + lane * (D * 4);
+#pragma unroll
+            for (int part = 0; part < D / 32; ++part)
+#pragma unroll
+              for (int c = 0; c < 32; c += 4)
+                st_shared_v4(rbuf + (32 * part + c) * 4, v[part][c], v[part][c + 1], v[part][c + 2], v[part][c + 3]);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              bulk_reduce_add_f32(base + (32 * wq) * D, wbuf, L::DQ_PART);
+              bulk_commit();
             }
+          }
         }
       }
     };
@@ -736,8 +754,9 @@ __global__ void __launch_bounds__(448, 1)
       drain(std::true_type{});
     } else {
       drain(std::false_type{});
-      // Let the TMA finish the last reductions before shared memory goes away.
-      if (L::DQ_T && warp == 8 && lane == 0) bulk_wait0();
+      // Let the TMA finish the last reductions before shared memory goes away
+      // (D = 128: warp 8 issued them; D = 64: lane 0 of each drain warp).
+      if (lane == 0 && (!L::DQ_T || warp == 8)) bulk_wait0();
     }
   }
 
