@@ -143,6 +143,14 @@ class ClockSampler:
                 "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
+def clock_peak_pct(fwd_tf, bwd_tf, clk):
+    mhz = clk.get("sm_mhz") if clk else None
+    if not mhz:
+        return None
+    peak = 148 * 8192 * mhz * 1e6 / 1e12
+    return {"fwd": 100 * fwd_tf / peak, "bwd": 100 * bwd_tf / peak, "peak": peak, "sm_mhz": mhz}
+
+
 def flops(w, causal):
     return w.fwd_flops(causal), w.bwd_flops(causal)
 
@@ -352,6 +360,12 @@ def run_ours(args, w, causal):
         "pct_of_nominal_2250": {"fwd": 100 * fwd_tf / NOMINAL_BF16_TFLOPS, "bwd": 100 * bwd_tf / NOMINAL_BF16_TFLOPS},
         "pct_of_measured_bf16": {"fwd": 100 * fwd_tf / peaks["bf16_tflops"], "bwd": 100 * bwd_tf / peaks["bf16_tflops"],
                                  "peak": peaks["bf16_tflops"]},
+        "pct_of_measured_bf16_sustained": {
+            "fwd": 100 * fwd_tf / peaks["bf16_tflops_sustained"], "bwd": 100 * bwd_tf / peaks["bf16_tflops_sustained"],
+            "peak": peaks["bf16_tflops_sustained"]},
+        # 148 SMs x 8192 dense bf16 FLOP per SM per clock (one M128 N128 K16
+        # tcgen05.mma every 64 cycles) at the SM clock sampled under load.
+        "pct_of_clock_peak": clock_peak_pct(fwd_tf, bwd_tf, clocks.summary()),
         "roofline": {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
                      "frac": achieved / peak_tf, "traffic": traffic,
                      "peak_source": f"{peaks_src} {'bf16_tflops_sustained' if sustained else 'bf16_tflops'}"},

@@ -90,7 +90,7 @@ def test_bwd_workloads_sampled(name):
     w = WORKLOADS[name]
     inp = make_inputs(w)
     dev = {n: inp[n].cuda() for n in ("q", "k", "v", "do")}
-    rows = sample_rows(w.S, 128, 118, w.seed)
+    rows = sample_rows(w.S, 128, 246 if name == "c5" else 118, w.seed)
     qn, kn, vn, don = (np64(inp[n]) for n in ("q", "k", "v", "do"))
     for causal in w.causal:
         o, lse = run_fwd(dev["q"], dev["k"], dev["v"], causal, w.scale)

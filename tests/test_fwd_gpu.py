@@ -81,7 +81,7 @@ def test_fwd_workloads_sampled(name):
     w = WORKLOADS[name]
     inp = make_inputs(w)
     q, k, v = inp["q"].cuda(), inp["k"].cuda(), inp["v"].cuda()
-    rows = sample_rows(w.S, 128, 118, w.seed)
+    rows = sample_rows(w.S, 128, 246 if name == "c5" else 118, w.seed)
     qn, kn, vn = np64(inp["q"]), np64(inp["k"]), np64(inp["v"])
     for causal in w.causal:
         o, lse = run_fwd(q, k, v, causal, w.scale)
