@@ -77,13 +77,23 @@ KERNEL_SOURCES = {
 }
 
 
+def _code_only(text: str) -> str:
+    """C++ source without comments and with whitespace collapsed, so that a
+    comment edit does not mark the kernel's counters stale."""
+    import re
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def kernel_source_hash(kernel: str) -> str:
-    """Hash of the sources a kernel is built from (to tell stale counters)."""
+    """Hash of the code of the sources a kernel is built from (to tell stale
+    counters)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "exact_io_aware_96_b200", "csrc")
     for name in KERNEL_SOURCES[kernel]:
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + f.read())
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            h.update(name.encode() + _code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

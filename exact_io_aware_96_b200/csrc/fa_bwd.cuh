@@ -31,8 +31,9 @@
 //               staged in shared memory a quarter (32 query rows) at a time
 //               and added by TMA bulk reductions, which keeps the reduction
 //               traffic off the load/store queues the softmax warps use.
-//               D = 64: red.global.add.v4 per query row. Deterministic mode:
-//               plain stores into the block's own slot.
+//               D = 64: each warp stages its 32 query rows (8 KB) and has the
+//               TMA add them. Deterministic mode: plain stores into the
+//               block's own slot.
 //   warp  12    TMA loader: K, V once; Q_i with lse2_i and dO_i with Dvec_i per
 //               query block, on separate rings (Q runs ahead of dO)
 //   warp  13    MMA issuer
