@@ -362,7 +362,12 @@ __global__ void __launch_bounds__(448, 1)
       }
     } else if (warp == kMmaWarp) {
       // ----------------------------------------------------------- MMA issuer
-      if (lane == 0 && n > 0) {
+      // The whole warp runs this loop converged; elect.sync picks the lane
+      // that issues each MMA and commit, and every wait is voted warp-wide.
+      if (n > 0) {
+        auto wait = [&](uint64_t* bar, uint32_t parity, int iter) {
+          return __all_sync(0xffffffffu, wait_bar(bar, parity, abort_flag, kRoleMma, iter));
+        };
         const uint32_t sK = smem_u32(smem + L::OFF_K);
         const uint32_t sV = smem_u32(smem + L::OFF_V);
         const uint32_t sQ = smem_u32(smem + L::OFF_Q);
@@ -382,23 +387,23 @@ __global__ void __launch_bounds__(448, 1)
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t o = (kk >> 2) * L::BLK + (kk & 3) * 32;
-            mma_ss(tmem + dcol, desc_add(a0, o), desc_add(b0, o), id_s, kk > 0);
+            mma_ss_w(tmem + dcol, desc_add(a0, o), desc_add(b0, o), id_s, kk > 0);
           }
         };
         const uint64_t ds_k = desc_sw128(sDS, 16, 1024);         // dS^T, K-major (A of dK)
         const uint64_t ds_mn = desc_sw128(sDS, L::BLK, 1024);    // dS^T, MN-major (dQ)
         const uint64_t k_mn = desc_sw128(sK, L::BLK, 1024);      // K, MN-major (dQ)
-        bool ok = wait_bar(kv_full, 0, abort_flag, kRoleMma, -1) && wait_bar(&q_full[0], 0, abort_flag, kRoleMma, 0);
+        bool ok = wait(kv_full, 0, -1) && wait(&q_full[0], 0, 0);
         if (ok) {
           tc_fence_after();
           issue_kt(L::COL_X, sK, sQ);
-          mma_commit(sx_full);
-          ok = wait_bar(&o_full[0], 0, abort_flag, kRoleMma, 0);
+          mma_commit_w(sx_full);
+          ok = wait(&o_full[0], 0, 0);
         }
         if (ok) {
           tc_fence_after();
           issue_kt(L::COL_Y, sV, sdO);
-          mma_commit(dp_full);
+          mma_commit_w(dp_full);
         }
         for (int i = 0; ok && i < n; ++i) {
           const int st = i % QS;
@@ -407,28 +412,28 @@ __global__ void __launch_bounds__(448, 1)
           const uint32_t qa = sQ + st * L::TILE;
           const uint64_t q_mn = desc_sw128(qa, L::BLK, 1024);
           const uint64_t do_mn = desc_sw128(sdO + ost * L::TILE, L::BLK, 1024);
-          if (!(ok = wait_bar(p_ready, ph, abort_flag, kRoleMma, i))) break;
+          if (!(ok = wait(p_ready, ph, i))) break;
           tc_fence_after();
           // dV += P^T dO
 #pragma unroll
           for (int kk = 0; kk < BM / 16; ++kk)
-            mma_ts(tmem + L::COL_DV, tmem + L::col_p(kk), desc_add(do_mn, kk * 2048), id_kv,
+            mma_ts_w(tmem + L::COL_DV, tmem + L::col_p(kk), desc_add(do_mn, kk * 2048), id_kv,
                    (i > 0 || kk > 0) ? 1u : 0u);
           if (i + 1 < n) {
             // S^T(i+1) into X as soon as dV(i) has been issued: X held only
             // P^T(i), which dV(i) reads first (the tensor pipe runs in issue
             // order). The softmax of block i+1 then overlaps dK(i) and dQ(i).
             const int sn = (i + 1) % QS;
-            if (!(ok = wait_bar(&q_full[sn], ((i + 1) / QS) & 1, abort_flag, kRoleMma, i + 1))) break;
+            if (!(ok = wait(&q_full[sn], ((i + 1) / QS) & 1, i + 1))) break;
             tc_fence_after();
             issue_kt(L::COL_X, sK, sQ + sn * L::TILE);
-            mma_commit(sx_full);
+            mma_commit_w(sx_full);
           }
-          if (!(ok = wait_bar(ds_ready, ph, abort_flag, kRoleMma, i))) break;
+          if (!(ok = wait(ds_ready, ph, i))) break;
           tc_fence_after();
           // dO(i) and Dvec(i) are free once dV(i) is done (the softmax warps
           // have read Dvec(i): ds_ready).
-          mma_commit(&o_empty[ost]);
+          mma_commit_w(&o_empty[ost]);
           // dQ (or dQ^T) into Y first, so that its drain overlaps dK(i): dP^T(i)
           // there has been read by the softmax warps.
 #pragma unroll
@@ -436,32 +441,32 @@ __global__ void __launch_bounds__(448, 1)
             const uint64_t dk_desc = desc_add(ds_mn, kk * 2048);
             const uint64_t k_desc = desc_add(k_mn, kk * 2048);
             if constexpr (L::DQ_T)
-              mma_ss(tmem + L::COL_Y, k_desc, dk_desc, id_q, kk > 0);
+              mma_ss_w(tmem + L::COL_Y, k_desc, dk_desc, id_q, kk > 0);
             else
-              mma_ss(tmem + L::COL_Y, dk_desc, k_desc, id_q, kk > 0);
+              mma_ss_w(tmem + L::COL_Y, dk_desc, k_desc, id_q, kk > 0);
           }
-          mma_commit(dq_full);
+          mma_commit_w(dq_full);
           // dK += dS^T Q, dS^T from shared memory (K-major: 128 keys x 128 queries)
 #pragma unroll
           for (int kk = 0; kk < BM / 16; ++kk) {
             const uint32_t o = (kk >> 2) * L::BLK + (kk & 3) * 32;
-            mma_ss(tmem + L::COL_DK, desc_add(ds_k, o), desc_add(q_mn, kk * 2048), id_kv,
+            mma_ss_w(tmem + L::COL_DK, desc_add(ds_k, o), desc_add(q_mn, kk * 2048), id_kv,
                    (i > 0 || kk > 0) ? 1u : 0u);
           }
-          mma_commit(&q_empty[st]);
-          mma_commit(ds_free);
+          mma_commit_w(&q_empty[st]);
+          mma_commit_w(ds_free);
           if (i + 1 < n) {
             // dP^T(i+1) into Y once dQ(i) has been read out of it.
             const int on = (i + 1) % L::OS;
-            if (!(ok = wait_bar(dq_free, ph, abort_flag, kRoleMma, i))) break;
-            if (!(ok = wait_bar(&o_full[on], ((i + 1) / L::OS) & 1, abort_flag, kRoleMma, i + 1))) break;
+            if (!(ok = wait(dq_free, ph, i))) break;
+            if (!(ok = wait(&o_full[on], ((i + 1) / L::OS) & 1, i + 1))) break;
             tc_fence_after();
             issue_kt(L::COL_Y, sV, sdO + on * L::TILE);
-            mma_commit(dp_full);
+            mma_commit_w(dp_full);
           }
         }
-        mma_commit(mma_done);
-        mma_commit(drain);
+        mma_commit_w(mma_done);
+        mma_commit_w(drain);
         drain_wait(drain, 0);
       }
     }

@@ -181,7 +181,12 @@ __global__ void __launch_bounds__(320, 1)
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && nmax > 0) {
+    // The whole warp runs this loop converged; elect.sync picks the lane that
+    // issues each MMA and commit, and every wait is voted warp-wide.
+    if (nmax > 0) {
+      auto wait = [&](uint64_t* bar, uint32_t parity, int iter) {
+        return __all_sync(0xffffffffu, wait_bar(bar, parity, abort_flag, kRoleMma, iter));
+      };
       const uint32_t idS = FP8 ? idesc_e4m3(128, 128, 0, 0) : idesc_f16(BF16, 128, 128, 0, 0);
       const uint32_t idO = FP8 ? idesc_e4m3(128, D, 0, 1) : idesc_f16(BF16, 128, D, 0, 1);
       const uint32_t sQ = smem_u32(smem + L::OFF_Q);
@@ -194,9 +199,9 @@ __global__ void __launch_bounds__(320, 1)
         for (int kk = 0; kk < L::RB / 32; ++kk) {  // 32 bytes of K per instruction
           const uint32_t o = (kk >> 2) * L::BLK + (kk & 3) * 32;
           if constexpr (FP8)
-            mma_ss_f8(tmem + t * 128, desc_add(qd, o), desc_add(kd, o), idS, kk > 0);
+            mma_ss_f8_w(tmem + t * 128, desc_add(qd, o), desc_add(kd, o), idS, kk > 0);
           else
-            mma_ss(tmem + t * 128, desc_add(qd, o), desc_add(kd, o), idS, kk > 0);
+            mma_ss_w(tmem + t * 128, desc_add(qd, o), desc_add(kd, o), idS, kk > 0);
         }
       };
       auto issue_PV = [&](int t, int st, int acc) {
@@ -206,22 +211,22 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
         for (int kk = 0; kk < (FP8 ? 4 : 8); ++kk) {
           if constexpr (FP8)
-            mma_ts_f8(tmem + 256 + t * D, tmem + t * 128 + kk * 8, desc_add(vd, kk * 4096), idO,
+            mma_ts_f8_w(tmem + 256 + t * D, tmem + t * 128 + kk * 8, desc_add(vd, kk * 4096), idO,
                       (acc || kk > 0) ? 1u : 0u);
           else
-            mma_ts(tmem + 256 + t * D, tmem + t * 128 + kk * 8, desc_add(vd, kk * 2048), idO,
+            mma_ts_w(tmem + 256 + t * D, tmem + t * 128 + kk * 8, desc_add(vd, kk * 2048), idO,
                    (acc || kk > 0) ? 1u : 0u);
         }
       };
-      bool ok = wait_bar(q_full, 0, abort_flag, kRoleMma, -1) && wait_bar(&k_full[0], 0, abort_flag, kRoleMma, 0);
+      bool ok = wait(q_full, 0, -1) && wait(&k_full[0], 0, 0);
       if (ok) {
         tc_fence_after();
         for (int t = 0; t < 2; ++t)
           if (nkv[t] > 0) {
             issue_S(t, 0);
-            mma_commit(&s_full[t]);
+            mma_commit_w(&s_full[t]);
           }
-        mma_commit(&k_empty[0]);
+        mma_commit_w(&k_empty[0]);
       }
       for (int j = 0; ok && j < nmax; ++j) {
         const int st = j % S;
@@ -229,30 +234,32 @@ __global__ void __launch_bounds__(320, 1)
         const int jn = j + 1;
         const int stn = jn % S;
         const uint32_t phn = (jn / S) & 1;
-        if (!(ok = wait_bar(&v_full[st], ph, abort_flag, kRoleMma, j))) break;
+        if (!(ok = wait(&v_full[st], ph, j))) break;
         bool kn_ready = false;
-        for (int t = 0; t < 2 && ok; ++t) {
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          if (!ok) break;
           if (j < nkv[t]) {
-            if (!(ok = wait_bar(&p_full[t], j & 1, abort_flag, kRoleMma, j))) break;
+            if (!(ok = wait(&p_full[t], j & 1, j))) break;
             tc_fence_after();
             issue_PV(t, st, j > 0);
-            if (j == nkv[t] - 1) mma_commit(&o_final[t]);
+            if (j == nkv[t] - 1) mma_commit_w(&o_final[t]);
           }
           if (jn < nkv[t]) {
             if (!kn_ready) {
-              if (!(ok = wait_bar(&k_full[stn], phn, abort_flag, kRoleMma, jn))) break;
+              if (!(ok = wait(&k_full[stn], phn, jn))) break;
               tc_fence_after();
               kn_ready = true;
             }
             issue_S(t, stn);
-            mma_commit(&s_full[t]);
+            mma_commit_w(&s_full[t]);
           }
         }
-        mma_commit(&v_empty[st]);
-        if (kn_ready) mma_commit(&k_empty[stn]);
+        mma_commit_w(&v_empty[st]);
+        if (kn_ready) mma_commit_w(&k_empty[stn]);
       }
-      // Wait for every MMA this thread issued before TMEM is released.
-      mma_commit(drain);
+      // Wait for every MMA this warp issued before TMEM is released.
+      mma_commit_w(drain);
       drain_wait(drain, 0);
     }
   } else {
