@@ -36,7 +36,7 @@
 //               block's own slot.
 //   warp  12    TMA loader: K, V once; Q_i with lse2_i and dO_i with Dvec_i per
 //               query block, on separate rings (Q runs ahead of dO)
-//   warp  13    MMA issuer
+//   warp  13    MMA issuer (the whole warp; elect.sync picks the issuing lane)
 // Blocks are 128 keys x 128 queries. Tensor memory: dK and dV accumulators,
 // X (S^T, then 16-bit P^T written back by the softmax warps and used as the
 // TMEM A operand of dV += P^T dO) and Y (dP^T, then dQ^T = K^T dS^T (D = 128)

@@ -12,7 +12,8 @@
 //   warps 0-3  softmax/epilogue for tile 0 (one query row per thread)
 //   warps 4-7  softmax/epilogue for tile 1
 //   warp  8    TMA loader: Q tiles once, then K_j and V_j into a ring
-//   warp  9    MMA issuer (one thread): S_t = Q_t K_j^T and O_t += P_t V_j
+//   warp  9    MMA issuer (the whole warp; elect.sync picks the issuing lane):
+//              S_t = Q_t K_j^T and O_t += P_t V_j
 // Tensor memory (512 columns x 128 lanes of fp32):
 //   [0,128) S_0   [128,256) S_1   [256,256+D) O_0   [256+D,256+2D) O_1
 //   P_t (16-bit) overwrites the first 64 columns of S_t and feeds PV as the
