@@ -3,7 +3,9 @@ plus ``forward``/``backward`` helpers that marshal torch CUDA tensors.
 
 Every computation runs in the library's kernels. There is no fallback: if
 libfa.so is missing, or a tensor is not a CUDA tensor, the call raises.
-torch is used only to allocate device memory and to name the stream.
+torch is used only to allocate device memory and to name the stream. The
+helpers check every buffer against the shapes that q and k imply (the C ABI
+receives only pointers and those sizes) and launch on q's device.
 """
 from __future__ import annotations
 
@@ -188,6 +190,33 @@ def _view(t: torch.Tensor) -> FaTensor:
     return FaTensor(t.data_ptr(), t.stride(0), t.stride(1), t.stride(2))
 
 
+def _expect(name: str, t: torch.Tensor, shape, dtype, device) -> None:
+    """The C ABI takes raw pointers and the sizes of q and k only, so every
+    other buffer must have exactly the shape, dtype and device they imply
+    (a smaller one would be read or written past its end)."""
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, q on {device}")
+
+
+def _expect_lse(lse: torch.Tensor, B: int, H: int, Sq: int, device) -> None:
+    _expect("lse", lse, (B, H, Sq), torch.float32, device)
+    if not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous fp32 [B, H, Sq] tensor")
+
+
+def _dims(q: torch.Tensor, k: torch.Tensor):
+    if q.dim() != 4 or k.dim() != 4:
+        raise ValueError("q and k must be [B, S, H, D] tensors")
+    B, Sq, H, D = q.shape
+    if (k.shape[0], k.shape[2], k.shape[3]) != (B, H, D):
+        raise ValueError(f"k: expected [B={B}, Sk, H={H}, D={D}], got {tuple(k.shape)}")
+    return B, Sq, H, D, k.shape[1]
+
+
 def _stream(stream) -> int:
     if stream is None:
         return torch.cuda.current_stream().cuda_stream
@@ -196,22 +225,23 @@ def _stream(stream) -> int:
 
 def forward(q, k, v, causal=False, scale=None, out=None, lse=None, stream=None):
     """O, LSE = attention(q, k, v) on [B, S, H, D] CUDA tensors (strided views allowed)."""
-    B, Sq, H, D = q.shape
-    Sk = k.shape[1]
+    B, Sq, H, D, Sk = _dims(q, k)
     dt = _dtype_code(q)
-    if k.dtype != q.dtype or v.dtype != q.dtype:
-        raise TypeError("q, k and v must share one dtype")
+    dev = q.device
+    _expect("k", k, (B, Sk, H, D), q.dtype, dev)
+    _expect("v", v, (B, Sk, H, D), q.dtype, dev)
     if scale is None:
         scale = D ** -0.5
     if out is None:
-        out = torch.empty((B, Sq, H, D), dtype=q.dtype, device=q.device)
+        out = torch.empty((B, Sq, H, D), dtype=q.dtype, device=dev)
     if lse is None:
-        lse = torch.empty((B, H, Sq), dtype=torch.float32, device=q.device)
-    if lse.dtype != torch.float32 or not lse.is_contiguous():
-        raise ValueError("lse must be a contiguous fp32 [B, H, Sq] tensor")
+        lse = torch.empty((B, H, Sq), dtype=torch.float32, device=dev)
+    _expect("out", out, (B, Sq, H, D), q.dtype, dev)
+    _expect_lse(lse, B, H, Sq, dev)
     p = FwdParams(_view(q), _view(k), _view(v), _view(out), lse.data_ptr(),
                   B, H, Sq, Sk, D, float(scale), int(bool(causal)), dt)
-    st = fa_fwd_ex(p, _stream(stream))
+    with torch.cuda.device(dev):
+        st = fa_fwd_ex(p, _stream(stream))
     if st != FA_OK:
         raise FaError(st, "fa_fwd_ex")
     return out, lse
@@ -222,26 +252,28 @@ def forward_fp8(q, k, v, q_descale, k_descale, v_descale, causal=False, scale=No
     """O, LSE from e4m3 tensors: the values attended over are q * q_descale,
     k * k_descale, v * v_descale. q, k, v are torch.float8_e4m3fn (or uint8
     holding E4M3 bytes) [B, S, H, D] CUDA views; O is ``out_dtype``."""
-    B, Sq, H, D = q.shape
-    Sk = k.shape[1]
-    for t in (q, k, v):
-        if t.dtype not in (torch.float8_e4m3fn, torch.uint8):
-            raise TypeError(f"e4m3 tensors (torch.float8_e4m3fn or uint8 bytes) only, got {t.dtype}")
+    B, Sq, H, D, Sk = _dims(q, k)
+    if q.dtype not in (torch.float8_e4m3fn, torch.uint8):
+        raise TypeError(f"e4m3 tensors (torch.float8_e4m3fn or uint8 bytes) only, got {q.dtype}")
+    dev = q.device
+    _expect("k", k, (B, Sk, H, D), q.dtype, dev)
+    _expect("v", v, (B, Sk, H, D), q.dtype, dev)
     od = _DT.get(out_dtype)
     if od is None:
         raise TypeError(f"out_dtype must be fp16 or bf16, got {out_dtype}")
     if scale is None:
         scale = D ** -0.5
     if out is None:
-        out = torch.empty((B, Sq, H, D), dtype=out_dtype, device=q.device)
+        out = torch.empty((B, Sq, H, D), dtype=out_dtype, device=dev)
     if lse is None:
-        lse = torch.empty((B, H, Sq), dtype=torch.float32, device=q.device)
-    if lse.dtype != torch.float32 or not lse.is_contiguous():
-        raise ValueError("lse must be a contiguous fp32 [B, H, Sq] tensor")
+        lse = torch.empty((B, H, Sq), dtype=torch.float32, device=dev)
+    _expect("out", out, (B, Sq, H, D), out_dtype, dev)
+    _expect_lse(lse, B, H, Sq, dev)
     p = FwdFp8Params(_view(q), _view(k), _view(v), _view(out), lse.data_ptr(),
                      B, H, Sq, Sk, D, float(scale), float(q_descale), float(k_descale), float(v_descale),
                      int(bool(causal)), od)
-    st = fa_fwd_fp8_ex(p, _stream(stream))
+    with torch.cuda.device(dev):
+        st = fa_fwd_fp8_ex(p, _stream(stream))
     if st != FA_OK:
         raise FaError(st, "fa_fwd_fp8_ex")
     return out, lse
@@ -260,20 +292,32 @@ def backward(q, k, v, o, lse, do, causal=False, scale=None, dq=None, dk=None, dv
     """dQ, dK, dV of L = sum(dO * O) for O = attention(q, k, v).
     ``deterministic=True`` sums dQ in a fixed order (bit-identical runs; more
     workspace and time)."""
-    B, Sq, H, D = q.shape
-    Sk = k.shape[1]
+    B, Sq, H, D, Sk = _dims(q, k)
     dt = _dtype_code(q)
+    dev = q.device
+    _expect("k", k, (B, Sk, H, D), q.dtype, dev)
+    _expect("v", v, (B, Sk, H, D), q.dtype, dev)
+    _expect("o", o, (B, Sq, H, D), q.dtype, dev)
+    _expect("do", do, (B, Sq, H, D), q.dtype, dev)
+    _expect_lse(lse, B, H, Sq, dev)
     if scale is None:
         scale = D ** -0.5
-    dq = torch.empty((B, Sq, H, D), dtype=q.dtype, device=q.device) if dq is None else dq
-    dk = torch.empty((B, Sk, H, D), dtype=q.dtype, device=q.device) if dk is None else dk
-    dv = torch.empty((B, Sk, H, D), dtype=q.dtype, device=q.device) if dv is None else dv
+    dq = torch.empty((B, Sq, H, D), dtype=q.dtype, device=dev) if dq is None else dq
+    dk = torch.empty((B, Sk, H, D), dtype=q.dtype, device=dev) if dk is None else dk
+    dv = torch.empty((B, Sk, H, D), dtype=q.dtype, device=dev) if dv is None else dv
+    _expect("dq", dq, (B, Sq, H, D), q.dtype, dev)
+    _expect("dk", dk, (B, Sk, H, D), q.dtype, dev)
+    _expect("dv", dv, (B, Sk, H, D), q.dtype, dev)
     if workspace is None:
-        workspace = workspace_for(B, H, Sq, D, q.device, Sk=Sk, deterministic=deterministic)
+        workspace = workspace_for(B, H, Sq, D, dev, Sk=Sk, deterministic=deterministic)
+    if workspace.device != dev or not workspace.is_contiguous():
+        raise ValueError(f"workspace must be a contiguous buffer on {dev}")
+    ws_bytes = workspace.numel() * workspace.element_size()
     p = BwdParams(_view(q), _view(k), _view(v), _view(o), _view(do), lse.data_ptr(),
                   _view(dq), _view(dk), _view(dv), B, H, Sq, Sk, D, float(scale),
-                  int(bool(causal)), dt, workspace.data_ptr(), workspace.numel(), int(bool(deterministic)))
-    st = fa_bwd_ex(p, _stream(stream))
+                  int(bool(causal)), dt, workspace.data_ptr(), ws_bytes, int(bool(deterministic)))
+    with torch.cuda.device(dev):
+        st = fa_bwd_ex(p, _stream(stream))
     if st != FA_OK:
         raise FaError(st, "fa_bwd_ex")
     return dq, dk, dv

@@ -170,3 +170,84 @@ def test_host_pipeline_needs_a_gpu():
         pytest.skip("a GPU is present")
     with pytest.raises(RuntimeError):
         HostAttentionPipeline(1, 128, 2, 64)
+
+
+def test_torch_helpers_check_every_buffer_against_q_and_k():
+    """The C ABI sizes everything from q and k; the helpers refuse any other
+    buffer whose shape, dtype or device differs (checked before the CUDA
+    check, so it runs on CPU tensors)."""
+    import torch
+    f16 = torch.float16
+    B, Sq, Sk, H, D = 1, 8, 12, 2, 64
+    q = torch.zeros(B, Sq, H, D, dtype=f16)
+    k = torch.zeros(B, Sk, H, D, dtype=f16)
+    v = torch.zeros(B, Sk, H, D, dtype=f16)
+    cases = [
+        (ValueError, "k: expected", dict(q=q, k=torch.zeros(B, Sk, H + 1, D, dtype=f16), v=v)),
+        (ValueError, "v: expected shape", dict(q=q, k=k, v=torch.zeros(B, Sk - 1, H, D, dtype=f16))),
+        (TypeError, "v: expected", dict(q=q, k=k, v=v.bfloat16())),
+        (ValueError, "out: expected shape", dict(q=q, k=k, v=v, out=torch.zeros(B, Sq - 1, H, D, dtype=f16))),
+        (TypeError, "out: expected", dict(q=q, k=k, v=v, out=torch.zeros(B, Sq, H, D, dtype=torch.bfloat16))),
+        (ValueError, "lse: expected shape", dict(q=q, k=k, v=v, lse=torch.zeros(B, Sq, H))),
+        (ValueError, "contiguous", dict(q=q, k=k, v=v, lse=torch.zeros(B, Sq, H).transpose(1, 2))),
+    ]
+    for exc, msg, kw in cases:
+        with pytest.raises(exc, match=msg):
+            fa.forward(**kw)
+    o = torch.zeros(B, Sq, H, D, dtype=f16)
+    lse = torch.zeros(B, H, Sq)
+    bwd_cases = [
+        (ValueError, "o: expected shape", dict(o=torch.zeros(B, Sk, H, D, dtype=f16))),
+        (TypeError, "do: expected", dict(do=o.bfloat16())),
+        (ValueError, "lse: expected shape", dict(lse=torch.zeros(B, H, Sk))),
+        (ValueError, "dq: expected shape", dict(dq=torch.zeros(B, Sk, H, D, dtype=f16))),
+        (ValueError, "dk: expected shape", dict(dk=torch.zeros(B, Sq, H, D, dtype=f16))),
+        (TypeError, "dv: expected", dict(dv=torch.zeros(B, Sk, H, D))),
+    ]
+    for exc, msg, kw in bwd_cases:
+        args = dict(q=q, k=k, v=v, o=o, lse=lse, do=o)
+        args.update(kw)
+        with pytest.raises(exc, match=msg):
+            fa.backward(**args)
+    # well-formed CPU tensors get as far as the device check
+    with pytest.raises(ValueError, match="CUDA device"):
+        fa.backward(q, k, v, o, lse, o, workspace=torch.zeros(16, dtype=torch.uint8))
+    u8 = torch.uint8
+    with pytest.raises(TypeError, match="k: expected"):
+        fa.forward_fp8(torch.zeros(B, Sq, H, D, dtype=u8), torch.zeros(B, Sk, H, D, dtype=torch.float8_e4m3fn),
+                       torch.zeros(B, Sk, H, D, dtype=u8), 1.0, 1.0, 1.0)
+    with pytest.raises(ValueError, match="v: expected shape"):
+        fa.forward_fp8(torch.zeros(B, Sq, H, D, dtype=u8), torch.zeros(B, Sk, H, D, dtype=u8),
+                       torch.zeros(B, Sq, H, D, dtype=u8), 1.0, 1.0, 1.0)
+
+
+def test_torch_helpers_marshal_well_formed_calls(monkeypatch):
+    """The argument marshalling of forward/backward/forward_fp8 for
+    well-formed buffers, with the device parts stubbed: the structs get the
+    sizes of q and k and the workspace size in bytes."""
+    import contextlib
+
+    import torch
+    seen = {}
+    monkeypatch.setattr(fa, "_view", lambda t: fa.FaTensor(0, t.stride(0), t.stride(1), t.stride(2)))
+    monkeypatch.setattr(fa, "_stream", lambda s: 0)
+    monkeypatch.setattr(torch.cuda, "device", lambda d: contextlib.nullcontext())
+    for name in ("fa_fwd_ex", "fa_fwd_fp8_ex", "fa_bwd_ex"):
+        monkeypatch.setattr(fa, name, lambda p, s, name=name: seen.__setitem__(name, p) or 0)
+    B, Sq, Sk, H, D = 2, 8, 12, 3, 64
+    q = torch.zeros(B, Sq, H, D, dtype=torch.bfloat16)
+    k = torch.zeros(B, Sk, H, D, dtype=torch.bfloat16)
+    o, lse = fa.forward(q, k, k.clone(), causal=True)
+    p = seen["fa_fwd_ex"]
+    assert (p.B, p.H, p.Sq, p.Sk, p.D, p.causal, p.dtype) == (B, H, Sq, Sk, D, 1, fa.FA_BF16)
+    assert o.shape == q.shape and lse.shape == (B, H, Sq)
+    ws = torch.zeros(100, dtype=torch.float32)
+    dq, dk, dv = fa.backward(q, k, k.clone(), o, lse, o.clone(), workspace=ws)
+    p = seen["fa_bwd_ex"]
+    assert (p.B, p.H, p.Sq, p.Sk, p.D, p.workspace_bytes) == (B, H, Sq, Sk, D, 400)
+    assert dq.shape == q.shape and dk.shape == k.shape and dv.shape == k.shape
+    q8 = torch.zeros(B, Sq, H, D, dtype=torch.uint8)
+    k8 = torch.zeros(B, Sk, H, D, dtype=torch.uint8)
+    o8, _ = fa.forward_fp8(q8, k8, k8.clone(), 0.5, 0.25, 2.0, out_dtype=torch.float16)
+    p = seen["fa_fwd_fp8_ex"]
+    assert (p.Sq, p.Sk, p.o_dtype, p.v_descale) == (Sq, Sk, fa.FA_FP16, 2.0) and o8.dtype == torch.float16
