@@ -1,0 +1,452 @@
+// fa_fwd_split.cuh — fused attention forward for sm_100a, 16-bit inputs, with
+// two softmax warpgroups per query tile.
+//
+// NOT BUILT INTO libfa.so YET: fa_api.cu does not include this header and no
+// entry point reaches it. It has been compiled for sm_100a (register and
+// spill counts) but never run on a GPU.
+//
+// Same computation and tensor-memory layout as fa_fwd.cuh (one CTA: two
+// 128-row query tiles of one (batch, head); S_t = Q_t K_j^T, the online
+// softmax in base 2 with a stale running max, O_t += P_t V_j, O divided by l
+// once, LSE stored; [P1] "性能引擎", [P2] item 2 "分块处理", [P4] §3.1-§3.2).
+// What changes is who runs the softmax: in fa_fwd.cuh one thread owns a
+// whole 128-key row of S_t; here two warpgroups share each row, one per
+// 64-key half, so a block's exponentials are spread over twice as many warps
+// and the softmax part of the per-tile chain (softmax of block j, then
+// P V(j) and S(j+1) on the tensor core) gets shorter.
+//
+// Warp roles (576 threads):
+//   warps 4g..4g+3, g = 2t + c: softmax of tile t, key half c (keys
+//              64c..64c+63 of each block), one query row per thread
+//   warp  16   TMA loader
+//   warp  17   MMA issuer (the whole warp; elect.sync picks the issuing lane)
+// Tensor memory (512 columns x 128 lanes of fp32), as in fa_fwd.cuh:
+//   [128t, 128t+128) S_t   [256+tD, 256+tD+D) O_t
+//   half c of S_t is columns 128t+64c .. +63; its P (16-bit, 32 columns)
+//   overwrites the first 32 of them, so each warpgroup only ever touches its
+//   own columns. P V(j) reads the two P halves from their two places.
+// Per block the two halves of a row agree on the running max: each stores
+// its partial row max in shared memory and arrives on the pair's mbarrier
+// (64 threads: the two warps that own the same 32 rows); after the wait both
+// take the larger value, so both follow the same m, raise decisions and
+// rescale factors. Each half rescales its own D/2 columns of O_t and keeps
+// its own partial sum l; the two sums are added in the epilogue through the
+// same exchange. Every wait is bounded (no named barriers), so an abort on
+// one side cannot leave the other waiting.
+//
+// Page legend: [P1] "Miniconda-Python3.9环境下使用FlashAttention优化训练";
+// [P2] "使用FlashAttention优化PyTorch模型注意力计算"; [P4] the FlashAttention-2
+// walkthrough titled "企业官网建设流程全解析".
+#pragma once
+
+#include "fa_common.cuh"
+#include "fa_fwd.cuh"  // fwd_kv_blocks
+
+namespace fa {
+
+template <int D>
+struct FwdSplitLayout {
+  static constexpr int kThreads = 576;
+  static constexpr int kLoaderWarp = 16;
+  static constexpr int kMmaWarp = 17;
+  static constexpr int KB = D / 64;              // 128-byte column blocks per row
+  static constexpr int TILE = 128 * D * 2;       // bytes of one 128-row tile
+  static constexpr int BLK = 128 * 128;          // one 128-row x 128-byte block
+  static constexpr int STAGES = (D == 128) ? 2 : 4;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + 2 * TILE;
+  static constexpr int OFF_V = OFF_K + STAGES * TILE;
+  // Partial row maxima, [block parity][tile][half][row], and partial sums,
+  // [tile][half][row].
+  static constexpr int OFF_PMAX = OFF_V + STAGES * TILE;
+  static constexpr int OFF_LSUM = OFF_PMAX + 2 * 2 * 2 * 128 * 4;
+  static constexpr int OFF_BAR = OFF_LSUM + 2 * 2 * 128 * 4;
+  // q_full, k_full/k_empty/v_full/v_empty[STAGES], s_full[2], p_full[2],
+  // o_final[2], pair[2][4], drain
+  static constexpr int NBAR = 1 + 4 * STAGES + 2 + 2 + 2 + 8 + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int BYTES = OFF_MISC + 16;
+  static constexpr int SMEM_ALLOC = BYTES + 1024;  // room to align the base to 1024
+  static constexpr int TMEM_COLS = 512;
+};
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(576, 1)
+    fa_fwd_split_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                        const __grid_constant__ CUtensorMap tmV, const FwdArgs a) {
+  using L = FwdSplitLayout<D>;
+  using namespace sm100;
+  constexpr int S = L::STAGES;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+  uint64_t* q_full = bars;
+  uint64_t* k_full = bars + 1;
+  uint64_t* k_empty = k_full + S;
+  uint64_t* v_full = k_empty + S;
+  uint64_t* v_empty = v_full + S;
+  uint64_t* s_full = v_empty + S;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* o_final = p_full + 2;
+  uint64_t* pair = o_final + 2;  // [t * 4 + quarter]
+  uint64_t* drain = pair + 8;
+  float* pmax = reinterpret_cast<float*>(smem + L::OFF_PMAX);
+  float* lsum = reinterpret_cast<float*>(smem + L::OFF_LSUM);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // Linear block order: all heads' heaviest query blocks first (causal).
+  const int hb_count = a.H * a.B;
+  const int rank = blockIdx.x / hb_count;
+  const int hb = blockIdx.x % hb_count;
+  const int h = hb % a.H;
+  const int b = hb / a.H;
+  const int qb = a.causal ? (a.n_qblocks - 1 - rank) : rank;
+  const int q0 = qb * 256;
+  int nkv[2];
+  nkv[0] = fwd_kv_blocks(q0, a.Sq, a.Sk, a.causal);
+  nkv[1] = fwd_kv_blocks(q0 + 128, a.Sq, a.Sk, a.causal);
+  const int nmax = max(nkv[0], nkv[1]);
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&s_full[t], 1);
+      mbar_init(&p_full[t], 256);
+      mbar_init(&o_final[t], 1);
+    }
+    for (int i = 0; i < 8; ++i) mbar_init(&pair[i], 64);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == L::kLoaderWarp && lane == 0) {
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+  }
+  if (warp == L::kMmaWarp) {
+    tmem_alloc(tmem_slot, L::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == L::kLoaderWarp) {
+    // ------------------------------------------------------------ loader
+    if (lane == 0 && nmax > 0) {
+      int q_bytes = 0;
+      for (int t = 0; t < 2; ++t) q_bytes += nkv[t] > 0 ? L::TILE : 0;
+      mbar_arrive_expect_tx(q_full, q_bytes);
+      for (int t = 0; t < 2; ++t)
+        if (nkv[t] > 0)
+          for (int kb = 0; kb < L::KB; ++kb)
+            tma_load_4d(smem + L::OFF_Q + t * L::TILE + kb * L::BLK, &tmQ, q_full, kb * 64, q0 + 128 * t, h, b);
+      int j = 0;
+      for (; j < nmax; ++j) {
+        const int st = j % S;
+        const uint32_t ph = (j / S) & 1;
+        if (!wait_bar(&k_empty[st], ph ^ 1, abort_flag, kRoleLoader, j)) break;
+        mbar_arrive_expect_tx(&k_full[st], L::TILE);
+        for (int kb = 0; kb < L::KB; ++kb)
+          tma_load_4d(smem + L::OFF_K + st * L::TILE + kb * L::BLK, &tmK, &k_full[st], kb * 64, j * 128, h, b);
+        if (!wait_bar(&v_empty[st], ph ^ 1, abort_flag, kRoleLoader, j)) {
+          ++j;  // K_j was issued
+          break;
+        }
+        mbar_arrive_expect_tx(&v_full[st], L::TILE);
+        for (int kb = 0; kb < L::KB; ++kb)
+          tma_load_4d(smem + L::OFF_V + st * L::TILE + kb * L::BLK, &tmV, &v_full[st], kb * 64, j * 128, h, b);
+      }
+      if (*abort_flag) {
+        // Let the copies already issued land before the CTA exits.
+        drain_wait(q_full, 0);
+        for (int i = max(0, j - S); i < j; ++i) {
+          drain_wait(&k_full[i % S], (i / S) & 1);
+          drain_wait(&v_full[i % S], (i / S) & 1);
+        }
+      }
+    }
+  } else if (warp == L::kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    if (nmax > 0) {
+      auto wait = [&](uint64_t* bar, uint32_t parity, int iter) {
+        return __all_sync(0xffffffffu, wait_bar(bar, parity, abort_flag, kRoleMma, iter));
+      };
+      const uint32_t idS = idesc_f16(BF16, 128, 128, 0, 0);
+      const uint32_t idO = idesc_f16(BF16, 128, D, 0, 1);
+      const uint32_t sQ = smem_u32(smem + L::OFF_Q);
+      const uint32_t sK = smem_u32(smem + L::OFF_K);
+      const uint32_t sV = smem_u32(smem + L::OFF_V);
+      auto issue_S = [&](int t, int st) {
+        const uint64_t qd = desc_sw128(sQ + t * L::TILE, 16, 1024);
+        const uint64_t kd = desc_sw128(sK + st * L::TILE, 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {  // 32 bytes of K per instruction
+          const uint32_t o = (kk >> 2) * L::BLK + (kk & 3) * 32;
+          mma_ss_w(tmem + t * 128, desc_add(qd, o), desc_add(kd, o), idS, kk > 0);
+        }
+      };
+      auto issue_PV = [&](int t, int st, int acc) {
+        const uint64_t vd = desc_sw128(sV + st * L::TILE, L::BLK, 1024);
+        // Keys 16kk..16kk+15: P of half kk >> 2 at columns 128t + 64(kk >> 2),
+        // 8 columns per 16 keys.
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts_w(tmem + 256 + t * D, tmem + t * 128 + 64 * (kk >> 2) + (kk & 3) * 8, desc_add(vd, kk * 2048), idO,
+                   (acc || kk > 0) ? 1u : 0u);
+      };
+      bool ok = wait(q_full, 0, -1) && wait(&k_full[0], 0, 0);
+      if (ok) {
+        tc_fence_after();
+        for (int t = 0; t < 2; ++t)
+          if (nkv[t] > 0) {
+            issue_S(t, 0);
+            mma_commit_w(&s_full[t]);
+          }
+        mma_commit_w(&k_empty[0]);
+      }
+      for (int j = 0; ok && j < nmax; ++j) {
+        const int st = j % S;
+        const uint32_t ph = (j / S) & 1;
+        const int jn = j + 1;
+        const int stn = jn % S;
+        const uint32_t phn = (jn / S) & 1;
+        if (!(ok = wait(&v_full[st], ph, j))) break;
+        bool kn_ready = false;
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          if (!ok) break;
+          if (j < nkv[t]) {
+            if (!(ok = wait(&p_full[t], j & 1, j))) break;
+            tc_fence_after();
+            issue_PV(t, st, j > 0);
+            if (j == nkv[t] - 1) mma_commit_w(&o_final[t]);
+          }
+          if (jn < nkv[t]) {
+            if (!kn_ready) {
+              if (!(ok = wait(&k_full[stn], phn, jn))) break;
+              tc_fence_after();
+              kn_ready = true;
+            }
+            issue_S(t, stn);
+            mma_commit_w(&s_full[t]);
+          }
+        }
+        mma_commit_w(&v_empty[st]);
+        if (kn_ready) mma_commit_w(&k_empty[stn]);
+      }
+      // Wait for every MMA this warp issued before TMEM is released.
+      mma_commit_w(drain);
+      drain_wait(drain, 0);
+    }
+  } else {
+    // ------------------------------------------------------- softmax / epilogue
+    const int g = warp >> 2;
+    const int t = g >> 1;        // query tile
+    const int c = g & 1;         // key half of every block
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;  // row within the tile
+    const int r0 = q0 + 128 * t;
+    const int row = r0 + r;
+    const int n = nkv[t];
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t tS = tmem + lane_base + t * 128 + 64 * c;          // this half's S, then P
+    const uint32_t tO = tmem + lane_base + 256 + t * D + c * (D / 2);  // this half's O columns
+    uint64_t* pbar = &pair[t * 4 + quarter];
+    const float sl2 = a.scale_log2;
+    const int off = a.Sk - a.Sq;
+    float m = -INFINITY;  // running max of x = s * scale * log2(e), the same in both halves
+    float l = 0.f;        // this half's running sum of 2^(x - m)
+    bool ok = true;
+
+    for (int j = 0; j < n; ++j) {
+      ok = __all_sync(0xffffffffu, wait_bar(&s_full[t], j & 1, abort_flag, kRoleSoftmax, j));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t rr[2][32];
+      tmem_ld32(tS, rr[0]);
+      tmem_ld32(tS + 32, rr[1]);
+      tmem_ld_wait();
+      reg_fence(rr[0]);
+      reg_fence(rr[1]);
+      float x[64];
+#pragma unroll
+      for (int q = 0; q < 2; ++q)
+#pragma unroll
+        for (int i = 0; i < 32; ++i) x[32 * q + i] = __uint_as_float(rr[q][i]);
+
+      const int k0 = j * 128 + 64 * c;  // first key of this half
+      const bool masked = k0 + 64 > a.Sk || (a.causal && k0 + 63 > r0 + off);
+      int lim = a.Sk - 1 - k0;  // last allowed column of this half
+      if (a.causal) lim = min(lim, row + off - k0);
+      if (masked) {
+#pragma unroll
+        for (int i = 0; i < 64; ++i) x[i] = (i <= lim) ? x[i] : -INFINITY;
+      }
+      float mx0 = max3(x[0], x[1], x[2]), mx1 = max3(x[3], x[4], x[5]);
+      float mx2 = max3(x[6], x[7], x[8]), mx3 = max3(x[9], x[10], x[11]);
+#pragma unroll
+      for (int i = 12; i < 60; i += 8) {
+        mx0 = max3(mx0, x[i], x[i + 1]);
+        mx1 = max3(mx1, x[i + 2], x[i + 3]);
+        mx2 = max3(mx2, x[i + 4], x[i + 5]);
+        mx3 = max3(mx3, x[i + 6], x[i + 7]);
+      }
+      mx0 = max3(mx0, x[60], x[61]);
+      mx1 = max3(mx1, x[62], x[63]);
+      const float pm = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+      // Exchange the partial maxima with the other half of the row. The slot
+      // of block j is rewritten in block j + 2, after the partner has passed
+      // the exchange of block j + 1 (which needs this thread's arrival).
+      float* slot = pmax + (((j & 1) * 2 + t) * 2) * 128;
+      slot[c * 128 + r] = pm;
+      mbar_arrive(pbar);
+      ok = __all_sync(0xffffffffu, wait_bar(pbar, j & 1, abort_flag, kRoleSoftmax, j));
+      if (!ok) break;
+      const float m_blk = fmaxf(pm, slot[(c ^ 1) * 128 + r]) * sl2;
+      const bool raise = m_blk > m + 8.0f;
+      float alpha = 1.f;
+      if (raise) {
+        alpha = ex2(m - m_blk);  // 0 when m was -inf
+        m = m_blk;
+      }
+      l *= alpha;
+      if (j > 0 && __any_sync(0xffffffffu, raise)) {
+        // Rescale this warp's 32 rows of this half's D/2 columns of O_t. P V(j-1)
+        // has completed: S(j) was issued after it and s_full(j) covers both.
+#pragma unroll 1
+        for (int q = 0; q < D / 64; ++q) {
+          uint32_t ov[32];
+          tmem_ld32(tO + 32 * q, ov);
+          tmem_ld_wait();
+          reg_fence(ov);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+          tmem_st32(tO + 32 * q, ov);
+        }
+      }
+      const float mu = (m == -INFINITY) ? 0.f : m;
+      // P = 2^(s * scale * log2e - m) for pairs of columns; one pair in four
+      // takes the polynomial exp2 on the FMA pipe, the rest the MUFU unit.
+      // The 64 S values are read again from tensor memory, 32 at a time, so
+      // that they need not stay in registers across the exchange: P of
+      // columns 0-31 goes to columns 0-15, P of 32-63 to 16-31, each after
+      // the S values under it have been read.
+      const uint64_t sl2x2 = f2(sl2, sl2);
+      const uint64_t negmu2 = f2(-mu, -mu);
+      uint64_t acc0 = f2(0.f, 0.f), acc1 = f2(0.f, 0.f);
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        uint32_t sv[32];
+        tmem_ld32(tS + 32 * q, sv);
+        tmem_ld_wait();
+        reg_fence(sv);
+        if (masked) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            sv[i] = (32 * q + i <= lim) ? sv[i] : __float_as_uint(-INFINITY);
+        }
+        uint32_t pw[16];
+#pragma unroll
+        for (int cc = 0; cc < 16; ++cc) {
+          const int p = 16 * q + cc;
+          const uint64_t tt =
+              fma2(f2(__uint_as_float(sv[2 * cc]), __uint_as_float(sv[2 * cc + 1])), sl2x2, negmu2);
+          uint64_t e;
+          if ((p & 3) == 3) {
+            e = exp2_poly2(tt);
+          } else {
+            float t0, t1;
+            f2_split(tt, t0, t1);
+            e = f2(ex2(t0), ex2(t1));
+          }
+          if (p & 1)
+            acc1 = add2(acc1, e);
+          else
+            acc0 = add2(acc0, e);
+          float e0, e1;
+          f2_split(e, e0, e1);
+          pw[cc] = pack2<BF16>(e0, e1);
+        }
+        tmem_st16(tS + 16 * q, pw);
+      }
+      {
+        const uint64_t acc = add2(acc0, acc1);
+        float a0, a1;
+        f2_split(acc, a0, a1);
+        l += a0 + a1;
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&p_full[t]);
+    }
+
+    // Epilogue: O = O_t / (l_0 + l_1), LSE = ln2 * (m + log2(l_0 + l_1)).
+    if (ok && !*abort_flag && r0 < a.Sq) {
+      const bool valid = row < a.Sq;
+      const int cb = c * (D / 2);  // first O column of this half
+      uint16_t* orow = reinterpret_cast<uint16_t*>(a.o) + static_cast<int64_t>(b) * a.o_sb +
+                       static_cast<int64_t>(row) * a.o_ss + static_cast<int64_t>(h) * a.o_sh;
+      if (n > 0) {
+        // The pair's barrier completed n phases in the loop; phase n carries l.
+        lsum[(t * 2 + c) * 128 + r] = l;
+        mbar_arrive(pbar);
+        if (__all_sync(0xffffffffu, wait_bar(pbar, n & 1, abort_flag, kRoleSoftmax, n)) &&
+            __all_sync(0xffffffffu, wait_bar(&o_final[t], 0, abort_flag, kRoleSoftmax, n))) {
+          const float lt = l + lsum[(t * 2 + (c ^ 1)) * 128 + r];
+          const bool has = (m != -INFINITY) && lt > 0.f;  // m stays -inf only for rows with no allowed key
+          const float inv_l = has ? a.o_scale / lt : 0.f;
+          tc_fence_after();
+#pragma unroll 1
+          for (int q = 0; q < D / 64; ++q) {
+            uint32_t ov[32];
+            tmem_ld32(tO + 32 * q, ov);
+            tmem_ld_wait();
+            reg_fence(ov);
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              pk[i] = pack2<BF16>(__uint_as_float(ov[2 * i]) * inv_l, __uint_as_float(ov[2 * i + 1]) * inv_l);
+            if (valid) {
+              uint4* dst = reinterpret_cast<uint4*>(orow + cb + 32 * q);
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                if (cb + 32 * q + 8 * i < a.d)
+                  dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+            }
+          }
+          if (valid && c == 0)
+            a.lse[(static_cast<int64_t>(b) * a.H + h) * a.Sq + row] =
+                has ? (m + __log2f(lt)) * 0.69314718055994531f : -INFINITY;
+        }
+      } else if (valid) {
+        uint4* dst = reinterpret_cast<uint4*>(orow);
+        for (int i = cb / 8; i < min(a.d, cb + D / 2) / 8; ++i) dst[i] = make_uint4(0, 0, 0, 0);
+        if (c == 0) a.lse[(static_cast<int64_t>(b) * a.H + h) * a.Sq + row] = -INFINITY;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == L::kMmaWarp) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, L::TMEM_COLS);
+  }
+}
+
+}  // namespace fa
