@@ -74,6 +74,7 @@ def max_over_ranks(x: float, device=None) -> float:
 KERNEL_SOURCES = {
     "fa_bwd": ["fa_bwd.cuh", "fa_common.cuh", "sm100.cuh"],
     "fa_fwd_kernel": ["fa_fwd.cuh", "fa_common.cuh", "sm100.cuh"],
+    "fa_fwd_split_kernel": ["fa_fwd_split.cuh", "fa_fwd.cuh", "fa_common.cuh", "sm100.cuh"],
 }
 
 
@@ -344,7 +345,7 @@ def run_ours(args, w, causal):
     if t_bwd >= t_fwd:
         dom, dom_flops, dom_t = "fa_bwd (fa_bwd_pre + fa_bwd_main + fa_bwd_dq)", fb, t_bwd_max / args.steps
     else:
-        dom, dom_flops, dom_t = "fa_fwd_kernel", ff, t_fwd_max / args.steps
+        dom, dom_flops, dom_t = "fa_fwd_split_kernel", ff, t_fwd_max / args.steps
     achieved = dom_flops / dom_t / 1e12
     traffic = None
     tpath = os.path.join(ROOT, "profiles", "traffic.json")

@@ -12,6 +12,7 @@
 
 #include "fa.h"
 #include "fa_fwd.cuh"
+#include "fa_fwd_split.cuh"
 #include "fa_bwd.cuh"
 
 namespace {
@@ -104,9 +105,9 @@ int prepare(F* fn, int smem_bytes, bool (&done)[kMaxDevices]) {
 
 template <int D, bool BF16>
 int launch_fwd(const fa_fwd_params* p, cudaStream_t stream) {
-  using L = fa::FwdLayout<D>;
+  using L = fa::FwdSplitLayout<D>;
   static bool done[kMaxDevices] = {};
-  auto* kern = &fa::fa_fwd_kernel<D, BF16>;
+  auto* kern = &fa::fa_fwd_split_kernel<D, BF16>;
   int st = prepare(kern, L::SMEM_ALLOC, done);
   if (st != FA_OK) return st;
   CUtensorMap mq, mk, mv;

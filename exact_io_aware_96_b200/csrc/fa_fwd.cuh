@@ -1,4 +1,7 @@
-// fa_fwd.cuh — fused attention forward for sm_100a.
+// fa_fwd.cuh — fused attention forward for sm_100a with one softmax
+// warpgroup per query tile; libfa.so runs it for e4m3 inputs (fa_fwd_fp8).
+// 16-bit inputs run the kernel of fa_fwd_split.cuh, which spreads each tile's
+// softmax over two warpgroups. fwd_kv_blocks below serves both.
 //
 // One CTA computes O and LSE for 256 query rows (two 128-row tiles, t = 0, 1)
 // of one (batch, head), streaming 128-key K/V blocks through shared memory:

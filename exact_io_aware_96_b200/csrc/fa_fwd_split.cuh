@@ -1,42 +1,61 @@
 // fa_fwd_split.cuh — fused attention forward for sm_100a, 16-bit inputs, with
 // two softmax warpgroups per query tile.
 //
-// NOT BUILT INTO libfa.so YET: fa_api.cu does not include this header and no
-// entry point reaches it. It has been compiled for sm_100a (register and
-// spill counts) but never run on a GPU.
+// One CTA computes O and LSE for 256 query rows (two 128-row tiles, t = 0, 1)
+// of one (batch, head), streaming 128-key K/V blocks through shared memory:
+// S_t = Q_t K_j^T, the online softmax and O_t += P_t V_j happen in one kernel
+// and the Sq x Sk score matrix never reaches device memory ([P1] "性能引擎":
+// the three steps fused into one kernel; [P2] item 2 "分块处理": tiles in
+// on-chip memory with an online softmax; [P5] "第三招": the next block is
+// prefetched while the current one is computed).
 //
-// Same computation and tensor-memory layout as fa_fwd.cuh (one CTA: two
-// 128-row query tiles of one (batch, head); S_t = Q_t K_j^T, the online
-// softmax in base 2 with a stale running max, O_t += P_t V_j, O divided by l
-// once, LSE stored; [P1] "性能引擎", [P2] item 2 "分块处理", [P4] §3.1-§3.2).
-// What changes is who runs the softmax: in fa_fwd.cuh one thread owns a
-// whole 128-key row of S_t; here two warpgroups share each row, one per
-// 64-key half, so a block's exponentials are spread over twice as many warps
-// and the softmax part of the per-tile chain (softmax of block j, then
-// P V(j) and S(j+1) on the tensor core) gets shorter.
+// Softmax per row in base 2: x = s * scale * log2(e), running max m and sum
+// l; the accumulator O_t stays unscaled and is divided by l once at the end,
+// and only LSE = ln2 * (m + log2 l) is stored ([P4] §3.1). The running max is
+// raised (and O_t, l rescaled) only when a block's max exceeds it by more than
+// 8, a factor 256; otherwise the stale max is kept, which is still exact
+// because l, O_t and LSE all use the same m.
+//
+// Per tile the work is a chain: softmax of block j, then P V(j) and S(j+1) on
+// the tensor core, then the softmax of block j + 1. The two tiles alternate,
+// so one tile's softmax runs while the tensor core works on the other's
+// products. Two warpgroups share every row of a tile, one per 64-key half of
+// each block, so a block's exponentials are spread over eight warps (two per
+// SM sub-partition) and the softmax link of the chain is short.
 //
 // Warp roles (576 threads):
-//   warps 4g..4g+3, g = 2t + c: softmax of tile t, key half c (keys
-//              64c..64c+63 of each block), one query row per thread
-//   warp  16   TMA loader
+//   warps 8t + 4c + r  softmax/epilogue of tile t, key half c (keys 64c ..
+//              64c + 63 of every block), TMEM lanes 32r .. 32r + 31, one query
+//              row per thread (r = warp % 4 is the warp's TMEM lane quarter)
+//   warp  16   TMA loader: Q tiles once, then K_j and V_j into a ring
 //   warp  17   MMA issuer (the whole warp; elect.sync picks the issuing lane)
-// Tensor memory (512 columns x 128 lanes of fp32), as in fa_fwd.cuh:
-//   [128t, 128t+128) S_t   [256+tD, 256+tD+D) O_t
-//   half c of S_t is columns 128t+64c .. +63; its P (16-bit, 32 columns)
-//   overwrites the first 32 of them, so each warpgroup only ever touches its
-//   own columns. P V(j) reads the two P halves from their two places.
-// Per block the two halves of a row agree on the running max: each stores
-// its partial row max in shared memory and arrives on the pair's mbarrier
-// (64 threads: the two warps that own the same 32 rows); after the wait both
-// take the larger value, so both follow the same m, raise decisions and
-// rescale factors. Each half rescales its own D/2 columns of O_t and keeps
-// its own partial sum l; the two sums are added in the epilogue through the
-// same exchange. Every wait is bounded (no named barriers), so an abort on
-// one side cannot leave the other waiting.
+// Tensor memory (512 columns x 128 lanes of fp32):
+//   [128t, 128t + 128) S_t   [256 + tD, 256 + tD + D) O_t
+//   Half c of S_t is columns 128t + 64c .. + 63; its P (16-bit, 32 columns)
+//   overwrites the first 32 of them, so each warpgroup only touches its own
+//   columns. P V(j) reads the two halves of P from their two places.
+// The two warps that own the same 32 rows of a tile (one per half) agree on
+// the running max once per block: each puts its partial row max in shared
+// memory and both meet at a 64-thread named barrier that also ANDs their
+// "still running" flags, so an abort seen by one side ends both sides at the
+// same point and neither waits for a partner that has left. Each half
+// rescales its own D/2 columns of O_t and keeps its own partial sum l; the two
+// sums meet the same way in the epilogue.
+//
+// Exponentials: 2^t on the MUFU unit (ex2.approx), except that on blocks
+// with no masked entry one pair in four goes through a polynomial on the FMA
+// pipe (sm100::exp2_poly2). Masked blocks use the MUFU unit for every entry,
+// so masked P entries are exactly 0.
+//
+// Work split over batch x heads x 256-row blocks ([P4] §3.2); for causal masks
+// the grid is ordered so the longest rows start first, key blocks past the
+// diagonal are skipped and only diagonal and tail blocks are masked element
+// by element ([P4] §4: causal skips about half the blocks).
 //
 // Page legend: [P1] "Miniconda-Python3.9环境下使用FlashAttention优化训练";
 // [P2] "使用FlashAttention优化PyTorch模型注意力计算"; [P4] the FlashAttention-2
-// walkthrough titled "企业官网建设流程全解析".
+// walkthrough titled "企业官网建设流程全解析"; [P5] the FlashAttention
+// "IO感知" overview (0539edu.com/news/165270).
 #pragma once
 
 #include "fa_common.cuh"
@@ -56,19 +75,54 @@ struct FwdSplitLayout {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + 2 * TILE;
   static constexpr int OFF_V = OFF_K + STAGES * TILE;
-  // Partial row maxima, [block parity][tile][half][row], and partial sums,
-  // [tile][half][row].
+  // Partial row maxima [block parity][tile][half][row] and partial sums
+  // [tile][half][row], fp32.
   static constexpr int OFF_PMAX = OFF_V + STAGES * TILE;
   static constexpr int OFF_LSUM = OFF_PMAX + 2 * 2 * 2 * 128 * 4;
   static constexpr int OFF_BAR = OFF_LSUM + 2 * 2 * 128 * 4;
   // q_full, k_full/k_empty/v_full/v_empty[STAGES], s_full[2], p_full[2],
-  // o_final[2], pair[2][4], drain
-  static constexpr int NBAR = 1 + 4 * STAGES + 2 + 2 + 2 + 8 + 1;
+  // o_final[2], drain
+  static constexpr int NBAR = 1 + 4 * STAGES + 2 + 2 + 2 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int SMEM_ALLOC = BYTES + 1024;  // room to align the base to 1024
   static constexpr int TMEM_COLS = 512;
 };
+
+// P = 2^(s * sl2 - mu) for 32 S values of one row (raw fp32 bits in sv),
+// packed to 16 words of two 16-bit values; adds the P values into acc0/acc1.
+// MASKED: entries past column `lim` are -inf (P = 0) and every exponential
+// runs on the MUFU unit, which returns exactly 0 for them.
+template <bool BF16, bool MASKED>
+__device__ __forceinline__ void fwd_exp32(const uint32_t (&sv)[32], int col0, int lim, uint64_t sl2x2,
+                                          uint64_t negmu2, uint64_t& acc0, uint64_t& acc1, uint32_t (&pw)[16]) {
+  using namespace sm100;
+#pragma unroll
+  for (int cc = 0; cc < 16; ++cc) {
+    float s0 = __uint_as_float(sv[2 * cc]);
+    float s1 = __uint_as_float(sv[2 * cc + 1]);
+    if constexpr (MASKED) {
+      s0 = (col0 + 2 * cc <= lim) ? s0 : -INFINITY;
+      s1 = (col0 + 2 * cc + 1 <= lim) ? s1 : -INFINITY;
+    }
+    const uint64_t tt = fma2(f2(s0, s1), sl2x2, negmu2);
+    uint64_t e;
+    if (!MASKED && (cc & 3) == 3) {
+      e = exp2_poly2(tt);
+    } else {
+      float t0, t1;
+      f2_split(tt, t0, t1);
+      e = f2(ex2(t0), ex2(t1));
+    }
+    if (cc & 1)
+      acc1 = add2(acc1, e);
+    else
+      acc0 = add2(acc0, e);
+    float e0, e1;
+    f2_split(e, e0, e1);
+    pw[cc] = pack2<BF16>(e0, e1);
+  }
+}
 
 template <int D, bool BF16>
 __global__ void __launch_bounds__(576, 1)
@@ -89,8 +143,7 @@ __global__ void __launch_bounds__(576, 1)
   uint64_t* s_full = v_empty + S;
   uint64_t* p_full = s_full + 2;
   uint64_t* o_final = p_full + 2;
-  uint64_t* pair = o_final + 2;  // [t * 4 + quarter]
-  uint64_t* drain = pair + 8;
+  uint64_t* drain = o_final + 2;
   float* pmax = reinterpret_cast<float*>(smem + L::OFF_PMAX);
   float* lsum = reinterpret_cast<float*>(smem + L::OFF_LSUM);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
@@ -122,10 +175,9 @@ __global__ void __launch_bounds__(576, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s_full[t], 1);
-      mbar_init(&p_full[t], 256);
+      mbar_init(&p_full[t], 8);  // one arrival per softmax warp of the tile
       mbar_init(&o_final[t], 1);
     }
-    for (int i = 0; i < 8; ++i) mbar_init(&pair[i], 64);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -171,7 +223,8 @@ __global__ void __launch_bounds__(576, 1)
           tma_load_4d(smem + L::OFF_V + st * L::TILE + kb * L::BLK, &tmV, &v_full[st], kb * 64, j * 128, h, b);
       }
       if (*abort_flag) {
-        // Let the copies already issued land before the CTA exits.
+        // Let the copies already issued land before the CTA exits. A V copy
+        // may be missing for the last K issued; its wait then runs out.
         drain_wait(q_full, 0);
         for (int i = max(0, j - S); i < j; ++i) {
           drain_wait(&k_full[i % S], (i / S) & 1);
@@ -181,12 +234,14 @@ __global__ void __launch_bounds__(576, 1)
     }
   } else if (warp == L::kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
+    // The whole warp runs this loop converged; elect.sync picks the lane that
+    // issues each MMA and commit, and every wait is voted warp-wide.
     if (nmax > 0) {
       auto wait = [&](uint64_t* bar, uint32_t parity, int iter) {
         return __all_sync(0xffffffffu, wait_bar(bar, parity, abort_flag, kRoleMma, iter));
       };
-      const uint32_t idS = idesc_f16(BF16, 128, 128, 0, 0);
-      const uint32_t idO = idesc_f16(BF16, 128, D, 0, 1);
+      constexpr uint32_t idS = idesc_f16(BF16, 128, 128, 0, 0);
+      constexpr uint32_t idO = idesc_f16(BF16, 128, D, 0, 1);
       const uint32_t sQ = smem_u32(smem + L::OFF_Q);
       const uint32_t sK = smem_u32(smem + L::OFF_K);
       const uint32_t sV = smem_u32(smem + L::OFF_V);
@@ -194,15 +249,15 @@ __global__ void __launch_bounds__(576, 1)
         const uint64_t qd = desc_sw128(sQ + t * L::TILE, 16, 1024);
         const uint64_t kd = desc_sw128(sK + st * L::TILE, 16, 1024);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {  // 32 bytes of K per instruction
+        for (int kk = 0; kk < D / 16; ++kk) {  // 32 bytes of the head dim per instruction
           const uint32_t o = (kk >> 2) * L::BLK + (kk & 3) * 32;
           mma_ss_w(tmem + t * 128, desc_add(qd, o), desc_add(kd, o), idS, kk > 0);
         }
       };
       auto issue_PV = [&](int t, int st, int acc) {
         const uint64_t vd = desc_sw128(sV + st * L::TILE, L::BLK, 1024);
-        // Keys 16kk..16kk+15: P of half kk >> 2 at columns 128t + 64(kk >> 2),
-        // 8 columns per 16 keys.
+        // Keys 16kk .. 16kk + 15: P of half kk >> 2 at columns 128t + 64(kk >> 2)
+        // + 8(kk & 3) (8 columns per 16 keys); V advances 16 rows of 128 bytes.
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_ts_w(tmem + 256 + t * D, tmem + t * 128 + 64 * (kk >> 2) + (kk & 3) * 8, desc_add(vd, kk * 2048), idO,
@@ -234,6 +289,10 @@ __global__ void __launch_bounds__(576, 1)
             tc_fence_after();
             issue_PV(t, st, j > 0);
             if (j == nkv[t] - 1) mma_commit_w(&o_final[t]);
+            // V_j is free once the last P V that reads it has run (tile 1's,
+            // or tile 0's where tile 1 has no block j): the loader may refill
+            // its stage while S(j+1) is still on the tensor core.
+            if (t == 1 || j >= nkv[1]) mma_commit_w(&v_empty[st]);
           }
           if (jn < nkv[t]) {
             if (!kn_ready) {
@@ -245,7 +304,6 @@ __global__ void __launch_bounds__(576, 1)
             mma_commit_w(&s_full[t]);
           }
         }
-        mma_commit_w(&v_empty[st]);
         if (kn_ready) mma_commit_w(&k_empty[stn]);
       }
       // Wait for every MMA this warp issued before TMEM is released.
@@ -254,18 +312,17 @@ __global__ void __launch_bounds__(576, 1)
     }
   } else {
     // ------------------------------------------------------- softmax / epilogue
-    const int g = warp >> 2;
-    const int t = g >> 1;        // query tile
-    const int c = g & 1;         // key half of every block
-    const int quarter = warp & 3;
+    const int t = warp >> 3;            // query tile
+    const int c = (warp >> 2) & 1;      // key half of every block
+    const int quarter = warp & 3;       // TMEM lane quarter
     const int r = quarter * 32 + lane;  // row within the tile
     const int r0 = q0 + 128 * t;
     const int row = r0 + r;
-    const int n = nkv[t];
+    const int n = t ? nkv[1] : nkv[0];
+    const int pair_bar = 1 + t * 4 + quarter;  // named barrier of the two warps that share these rows
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t tS = tmem + lane_base + t * 128 + 64 * c;          // this half's S, then P
+    const uint32_t tS = tmem + lane_base + t * 128 + 64 * c;          // this half's S, then its P
     const uint32_t tO = tmem + lane_base + 256 + t * D + c * (D / 2);  // this half's O columns
-    uint64_t* pbar = &pair[t * 4 + quarter];
     const float sl2 = a.scale_log2;
     const int off = a.Sk - a.Sq;
     float m = -INFINITY;  // running max of x = s * scale * log2(e), the same in both halves
@@ -273,49 +330,53 @@ __global__ void __launch_bounds__(576, 1)
     bool ok = true;
 
     for (int j = 0; j < n; ++j) {
-      ok = __all_sync(0xffffffffu, wait_bar(&s_full[t], j & 1, abort_flag, kRoleSoftmax, j));
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t rr[2][32];
-      tmem_ld32(tS, rr[0]);
-      tmem_ld32(tS + 32, rr[1]);
-      tmem_ld_wait();
-      reg_fence(rr[0]);
-      reg_fence(rr[1]);
-      float x[64];
-#pragma unroll
-      for (int q = 0; q < 2; ++q)
-#pragma unroll
-        for (int i = 0; i < 32; ++i) x[32 * q + i] = __uint_as_float(rr[q][i]);
-
+      const bool ready = __all_sync(0xffffffffu, wait_bar(&s_full[t], j & 1, abort_flag, kRoleSoftmax, j));
       const int k0 = j * 128 + 64 * c;  // first key of this half
       const bool masked = k0 + 64 > a.Sk || (a.causal && k0 + 63 > r0 + off);
       int lim = a.Sk - 1 - k0;  // last allowed column of this half
       if (a.causal) lim = min(lim, row + off - k0);
-      if (masked) {
-#pragma unroll
-        for (int i = 0; i < 64; ++i) x[i] = (i <= lim) ? x[i] : -INFINITY;
-      }
-      float mx0 = max3(x[0], x[1], x[2]), mx1 = max3(x[3], x[4], x[5]);
-      float mx2 = max3(x[6], x[7], x[8]), mx3 = max3(x[9], x[10], x[11]);
-#pragma unroll
-      for (int i = 12; i < 60; i += 8) {
-        mx0 = max3(mx0, x[i], x[i + 1]);
-        mx1 = max3(mx1, x[i + 2], x[i + 3]);
-        mx2 = max3(mx2, x[i + 4], x[i + 5]);
-        mx3 = max3(mx3, x[i + 6], x[i + 7]);
-      }
-      mx0 = max3(mx0, x[60], x[61]);
-      mx1 = max3(mx1, x[62], x[63]);
-      const float pm = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
-      // Exchange the partial maxima with the other half of the row. The slot
-      // of block j is rewritten in block j + 2, after the partner has passed
-      // the exchange of block j + 1 (which needs this thread's arrival).
       float* slot = pmax + (((j & 1) * 2 + t) * 2) * 128;
-      slot[c * 128 + r] = pm;
-      mbar_arrive(pbar);
-      ok = __all_sync(0xffffffffu, wait_bar(pbar, j & 1, abort_flag, kRoleSoftmax, j));
-      if (!ok) break;
+      float pm = -INFINITY;
+      if (ready) {
+        tc_fence_after();
+        uint32_t rr[2][32];
+        tmem_ld32(tS, rr[0]);
+        tmem_ld32(tS + 32, rr[1]);
+        tmem_ld_wait();
+        reg_fence(rr[0]);
+        reg_fence(rr[1]);
+        float x[64];
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+#pragma unroll
+          for (int i = 0; i < 32; ++i) x[32 * q + i] = __uint_as_float(rr[q][i]);
+        if (masked) {
+#pragma unroll
+          for (int i = 0; i < 64; ++i) x[i] = (i <= lim) ? x[i] : -INFINITY;
+        }
+        float mx0 = max3(x[0], x[1], x[2]), mx1 = max3(x[3], x[4], x[5]);
+        float mx2 = max3(x[6], x[7], x[8]), mx3 = max3(x[9], x[10], x[11]);
+#pragma unroll
+        for (int i = 12; i < 60; i += 8) {
+          mx0 = max3(mx0, x[i], x[i + 1]);
+          mx1 = max3(mx1, x[i + 2], x[i + 3]);
+          mx2 = max3(mx2, x[i + 4], x[i + 5]);
+          mx3 = max3(mx3, x[i + 6], x[i + 7]);
+        }
+        mx0 = max3(mx0, x[60], x[61]);
+        mx1 = max3(mx1, x[62], x[63]);
+        pm = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+        // The slot of block j is written again in block j + 2, after the
+        // partner has passed the barrier of block j + 1, i.e. after it has
+        // read this value.
+        slot[c * 128 + r] = pm;
+      }
+      // Both warps of the pair reach this barrier in every block, running or
+      // not; it publishes the partial maxima and ANDs the two "ready" flags.
+      if (!named_bar_and(pair_bar, 64, ready)) {
+        ok = false;
+        break;
+      }
       const float m_blk = fmaxf(pm, slot[(c ^ 1) * 128 + r]) * sl2;
       const bool raise = m_blk > m + 8.0f;
       float alpha = 1.f;
@@ -325,8 +386,9 @@ __global__ void __launch_bounds__(576, 1)
       }
       l *= alpha;
       if (j > 0 && __any_sync(0xffffffffu, raise)) {
-        // Rescale this warp's 32 rows of this half's D/2 columns of O_t. P V(j-1)
-        // has completed: S(j) was issued after it and s_full(j) covers both.
+        // Rescale this warp's 32 rows of this half's D/2 columns of O_t.
+        // P V(j-1) has completed: S(j) was issued after it and s_full(j)
+        // covers both.
 #pragma unroll 1
         for (int q = 0; q < D / 64; ++q) {
           uint32_t ov[32];
@@ -339,48 +401,24 @@ __global__ void __launch_bounds__(576, 1)
         }
       }
       const float mu = (m == -INFINITY) ? 0.f : m;
-      // P = 2^(s * scale * log2e - m) for pairs of columns; one pair in four
-      // takes the polynomial exp2 on the FMA pipe, the rest the MUFU unit.
-      // The 64 S values are read again from tensor memory, 32 at a time, so
-      // that they need not stay in registers across the exchange: P of
-      // columns 0-31 goes to columns 0-15, P of 32-63 to 16-31, each after
-      // the S values under it have been read.
       const uint64_t sl2x2 = f2(sl2, sl2);
       const uint64_t negmu2 = f2(-mu, -mu);
       uint64_t acc0 = f2(0.f, 0.f), acc1 = f2(0.f, 0.f);
+      // S is read again from tensor memory 32 columns at a time, so the 64 S
+      // values need not stay in registers across the exchange: P of columns
+      // 0-31 goes to columns 0-15, P of 32-63 to 16-31, each after the S
+      // values under it have been read.
 #pragma unroll
       for (int q = 0; q < 2; ++q) {
         uint32_t sv[32];
         tmem_ld32(tS + 32 * q, sv);
         tmem_ld_wait();
         reg_fence(sv);
-        if (masked) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            sv[i] = (32 * q + i <= lim) ? sv[i] : __float_as_uint(-INFINITY);
-        }
         uint32_t pw[16];
-#pragma unroll
-        for (int cc = 0; cc < 16; ++cc) {
-          const int p = 16 * q + cc;
-          const uint64_t tt =
-              fma2(f2(__uint_as_float(sv[2 * cc]), __uint_as_float(sv[2 * cc + 1])), sl2x2, negmu2);
-          uint64_t e;
-          if ((p & 3) == 3) {
-            e = exp2_poly2(tt);
-          } else {
-            float t0, t1;
-            f2_split(tt, t0, t1);
-            e = f2(ex2(t0), ex2(t1));
-          }
-          if (p & 1)
-            acc1 = add2(acc1, e);
-          else
-            acc0 = add2(acc0, e);
-          float e0, e1;
-          f2_split(e, e0, e1);
-          pw[cc] = pack2<BF16>(e0, e1);
-        }
+        if (masked)
+          fwd_exp32<BF16, true>(sv, 32 * q, lim, sl2x2, negmu2, acc0, acc1, pw);
+        else
+          fwd_exp32<BF16, false>(sv, 32 * q, lim, sl2x2, negmu2, acc0, acc1, pw);
         tmem_st16(tS + 16 * q, pw);
       }
       {
@@ -391,24 +429,25 @@ __global__ void __launch_bounds__(576, 1)
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&p_full[t]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[t]);
     }
 
     // Epilogue: O = O_t / (l_0 + l_1), LSE = ln2 * (m + log2(l_0 + l_1)).
-    if (ok && !*abort_flag && r0 < a.Sq) {
+    // Both warps of the pair arrive here with the same `ok` (the loop's
+    // barrier ANDs it), so both take the barrier below or neither does.
+    if (ok && r0 < a.Sq) {
+      lsum[(t * 2 + c) * 128 + r] = l;
+      const bool go = named_bar_and(pair_bar, 64, !*abort_flag);
       const bool valid = row < a.Sq;
       const int cb = c * (D / 2);  // first O column of this half
       uint16_t* orow = reinterpret_cast<uint16_t*>(a.o) + static_cast<int64_t>(b) * a.o_sb +
                        static_cast<int64_t>(row) * a.o_ss + static_cast<int64_t>(h) * a.o_sh;
-      if (n > 0) {
-        // The pair's barrier completed n phases in the loop; phase n carries l.
-        lsum[(t * 2 + c) * 128 + r] = l;
-        mbar_arrive(pbar);
-        if (__all_sync(0xffffffffu, wait_bar(pbar, n & 1, abort_flag, kRoleSoftmax, n)) &&
-            __all_sync(0xffffffffu, wait_bar(&o_final[t], 0, abort_flag, kRoleSoftmax, n))) {
-          const float lt = l + lsum[(t * 2 + (c ^ 1)) * 128 + r];
-          const bool has = (m != -INFINITY) && lt > 0.f;  // m stays -inf only for rows with no allowed key
-          const float inv_l = has ? a.o_scale / lt : 0.f;
+      if (go && n > 0) {
+        const float lt = l + lsum[(t * 2 + (c ^ 1)) * 128 + r];
+        const bool has = (m != -INFINITY) && lt > 0.f;  // m stays -inf only for rows with no allowed key
+        const float inv_l = has ? a.o_scale / lt : 0.f;
+        if (__all_sync(0xffffffffu, wait_bar(&o_final[t], 0, abort_flag, kRoleSoftmax, n))) {
           tc_fence_after();
 #pragma unroll 1
           for (int q = 0; q < D / 64; ++q) {
@@ -432,7 +471,8 @@ __global__ void __launch_bounds__(576, 1)
             a.lse[(static_cast<int64_t>(b) * a.H + h) * a.Sq + row] =
                 has ? (m + __log2f(lt)) * 0.69314718055994531f : -INFINITY;
         }
-      } else if (valid) {
+      } else if (go && valid) {
+        // No key reaches these rows: O = 0, LSE = -inf.
         uint4* dst = reinterpret_cast<uint4*>(orow);
         for (int i = cb / 8; i < min(a.d, cb + D / 2) / 8; ++i) dst[i] = make_uint4(0, 0, 0, 0);
         if (c == 0) a.lse[(static_cast<int64_t>(b) * a.H + h) * a.Sq + row] = -INFINITY;
