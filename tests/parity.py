@@ -44,11 +44,45 @@ def rel_l2(a, b):
     return np.linalg.norm(a - b) / (nb if nb > 0 else 1.0)
 
 
-def check_grad(g_gpu, g_ref, what=""):
+def blocks_rel_l2(a, b, row_axis, head_axes=(), block=128, rows=None, floor=1e-3):
+    """Relative L2 error of every (head, 128-row block) piece of ``a`` against
+    ``b``: ||a_p - b_p|| / max(||b_p||, f_p), where f_p = floor * ||b|| *
+    sqrt(size_p / size) is a small fraction of the piece's share of the whole
+    norm (it only matters for pieces whose reference is, by cancellation,
+    almost zero). ``rows`` gives the sequence index of each position along
+    ``row_axis`` (default 0, 1, ...; sampled rows are grouped by the block
+    they fall in). Yields ((head indices, first row of the block), error)."""
+    a, b = np.asarray(a, np.float64), np.asarray(b, np.float64)
+    nb_all = np.linalg.norm(b)
+    n = a.shape[row_axis]
+    blk = (np.arange(n) if rows is None else np.asarray(rows)) // block
+    heads = [a.shape[ax] for ax in head_axes]
+    for idx in np.ndindex(*heads):
+        for kb in np.unique(blk):
+            sl = [slice(None)] * a.ndim
+            sl[row_axis] = np.nonzero(blk == kb)[0]
+            for ax, i in zip(head_axes, idx):
+                sl[ax] = i
+            pa, pb = a[tuple(sl)], b[tuple(sl)]
+            share = nb_all * np.sqrt(pb.size / b.size) if b.size else 0.0
+            den = max(np.linalg.norm(pb), floor * share)
+            err = np.linalg.norm(pa - pb) / den if den > 0 else np.linalg.norm(pa - pb)
+            yield (idx, int(kb) * block), float(err)
+
+
+def check_grad(g_gpu, g_ref, what="", row_axis=None, head_axes=(), rows=None):
+    """Relative L2 error <= GRAD_TOL over the whole tensor and, when
+    ``row_axis`` is given, over every head and every 128-row block along that
+    axis (the same bar applied piece by piece, so that an error confined to
+    one block or one head cannot hide in the norm of the rest)."""
     g_gpu = np.asarray(g_gpu, np.float64)
     assert np.all(np.isfinite(g_gpu)), f"{what}: non-finite gradient"
     e = rel_l2(g_gpu, g_ref)
     assert e <= GRAD_TOL, f"{what}: relative L2 error {e:.3e} > {GRAD_TOL}"
+    if row_axis is not None:
+        worst = max(blocks_rel_l2(g_gpu, g_ref, row_axis, head_axes, rows=rows), key=lambda x: x[1])
+        assert worst[1] <= GRAD_TOL, (f"{what}: relative L2 error {worst[1]:.3e} > {GRAD_TOL} in the piece "
+                                      f"(head index {worst[0][0]}, rows from {worst[0][1]})")
     return e
 
 
@@ -83,7 +117,7 @@ def full_check(inp_cpu, causal, scale=None, backward=True, what=""):
     dq, dk, dv = run_bwd(dev["q"], dev["k"], dev["v"], o, lse, dev["do"], causal, sc)
     dq_r, dk_r, dv_r, _ = oracle.attention_backward(np64(q), np64(k), np64(v), np64(do), sc, causal)
     for name, g, r in (("dq", dq, dq_r), ("dk", dk, dk_r), ("dv", dv, dv_r)):
-        check_grad(np64(g), r, f"{what} {name}")
+        check_grad(np64(g), r, f"{what} {name}", row_axis=1, head_axes=(0, 2))
 
 
 # ------------------------------------------------------------------ e4m3 forward

@@ -26,7 +26,7 @@ def test_flash_attn_func_backward(causal, D, dtype):
     assert np.max(np.abs(np64(o) - o_ref)) <= (1e-2 if dtype == torch.float16 else 2e-2)
     dq_r, dk_r, dv_r, _ = oracle.attention_backward(np64(c["q"]), np64(c["k"]), np64(c["v"]), np64(c["do"]), sc, causal)
     for g, r, name in ((q.grad, dq_r, "dq"), (k.grad, dk_r, "dk"), (v.grad, dv_r, "dv")):
-        check_grad(np64(g), r, name)
+        check_grad(np64(g), r, name, row_axis=1, head_axes=(0, 2))
 
 
 def test_qkvpacked_usage_snippet():
@@ -46,7 +46,7 @@ def test_qkvpacked_usage_snippet():
     dq_r, dk_r, dv_r, _ = oracle.attention_backward(qn, kn, vn, ones, w.scale, False)
     g = np64(qkv.grad)
     for j, r in enumerate((dq_r, dk_r, dv_r)):
-        check_grad(g[:, :, j], r, f"dqkv[{j}]")
+        check_grad(g[:, :, j], r, f"dqkv[{j}]", row_axis=1, head_axes=(0, 2))
 
 
 def test_module_and_noncontiguous_inputs():
@@ -116,4 +116,4 @@ def test_flash_attn_func_deterministic():
         assert torch.equal(a, b)
     dq_r, _, _, _ = oracle.attention_backward(np64(c["q"]), np64(c["k"]), np64(c["v"]), np64(c["do"]),
                                               128 ** -0.5, True)
-    check_grad(np64(grads[0][0]), dq_r, "dq")
+    check_grad(np64(grads[0][0]), dq_r, "dq", row_axis=1, head_axes=(0, 2))

@@ -69,7 +69,7 @@ def test_bwd_packed_qkv():
     dq_r, dk_r, dv_r, _ = oracle.attention_backward(qn, kn, vn, don, w.scale, False)
     g = np64(dqkv)
     for j, (name, ref) in enumerate((("dq", dq_r), ("dk", dk_r), ("dv", dv_r))):
-        check_grad(g[:, :, j], ref, f"c2 {name}")
+        check_grad(g[:, :, j], ref, f"c2 {name}", row_axis=1, head_axes=(0, 2))
 
 
 def test_bwd_repeatable_dk_dv():
@@ -100,11 +100,12 @@ def test_bwd_workloads_sampled(name):
         for h in range(w.H):
             got.append(dq[0, rows, h])
             ref.append(oracle.attention_backward_dq_rows(qn, kn, vn, don, w.scale, causal, 0, h, rows))
-        check_grad(np.stack(got), np.stack(ref), f"{name} dq rows causal={causal}")
+        check_grad(np.stack(got), np.stack(ref), f"{name} dq rows causal={causal}",
+                   row_axis=1, head_axes=(0,), rows=rows)
         for h in (0, w.H - 1):
             hd = oracle.attention_head(qn, kn, vn, don, w.scale, causal, 0, h)
-            check_grad(dk[0, :, h], hd["dk"], f"{name} dk h{h} causal={causal}")
-            check_grad(dv[0, :, h], hd["dv"], f"{name} dv h{h} causal={causal}")
+            check_grad(dk[0, :, h], hd["dk"], f"{name} dk h{h} causal={causal}", row_axis=0)
+            check_grad(dv[0, :, h], hd["dv"], f"{name} dv h{h} causal={causal}", row_axis=0)
             del hd
 
 
@@ -124,7 +125,7 @@ def _det_case(c, causal, scale=None, what=""):
     qn, kn, vn, don = (np64(c[n]) for n in ("q", "k", "v", "do"))
     dq_r, dk_r, dv_r, _ = oracle.attention_backward(qn, kn, vn, don, sc, causal)
     for name, g, r in (("dq", dq1, dq_r), ("dk", dk1, dk_r), ("dv", dv1, dv_r)):
-        check_grad(np64(g), r, f"{what} det {name}")
+        check_grad(np64(g), r, f"{what} det {name}", row_axis=1, head_axes=(0, 2))
     # the atomic path sums the same fp32 blocks in another order
     dqa, dka, dva = run_bwd(q, k, v, o, lse, do, causal, sc)
     assert torch.equal(dka, dk1) and torch.equal(dva, dv1)
@@ -170,4 +171,4 @@ def test_bwd_deterministic_c4_full_size():
     qn, kn, vn, don = (np64(inp[n]) for n in ("q", "k", "v", "do"))
     got = np.stack([np64(dq1)[0, rows, h] for h in (0, w.H - 1)])
     ref = np.stack([oracle.attention_backward_dq_rows(qn, kn, vn, don, w.scale, True, 0, h, rows) for h in (0, w.H - 1)])
-    check_grad(got, ref, "c4 det dq rows")
+    check_grad(got, ref, "c4 det dq rows", row_axis=1, head_axes=(0,), rows=rows)
