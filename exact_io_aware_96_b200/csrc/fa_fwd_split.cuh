@@ -81,8 +81,8 @@ struct FwdSplitLayout {
   static constexpr int OFF_LSUM = OFF_PMAX + 2 * 2 * 2 * 128 * 4;
   static constexpr int OFF_BAR = OFF_LSUM + 2 * 2 * 128 * 4;
   // q_full, k_full/k_empty/v_full/v_empty[STAGES], s_full[2], p_full[2],
-  // o_final[2], drain
-  static constexpr int NBAR = 1 + 4 * STAGES + 2 + 2 + 2 + 1;
+  // o_final[2], drain, pv_done[2]
+  static constexpr int NBAR = 1 + 4 * STAGES + 2 + 2 + 2 + 1 + 2;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int SMEM_ALLOC = BYTES + 1024;  // room to align the base to 1024
@@ -131,6 +131,11 @@ __global__ void __launch_bounds__(576, 1)
   using L = FwdSplitLayout<D>;
   using namespace sm100;
   constexpr int S = L::STAGES;
+  // D = 64 leaves room in TMEM for a third S buffer: S products rotate over
+  // three buffers (see the MMA issuer), so a tile's next S is ready before
+  // its softmax finishes the current block.
+  constexpr bool kRot3 = (D == 64);
+  constexpr int OBASE = kRot3 ? 384 : 256;  // first TMEM column of O_0
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -144,6 +149,7 @@ __global__ void __launch_bounds__(576, 1)
   uint64_t* p_full = s_full + 2;
   uint64_t* o_final = p_full + 2;
   uint64_t* drain = o_final + 2;
+  uint64_t* pv_done = drain + 1;  // D = 64: P_t(j) V_j has completed
   float* pmax = reinterpret_cast<float*>(smem + L::OFF_PMAX);
   float* lsum = reinterpret_cast<float*>(smem + L::OFF_LSUM);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
@@ -177,6 +183,7 @@ __global__ void __launch_bounds__(576, 1)
       mbar_init(&s_full[t], 1);
       mbar_init(&p_full[t], 8);  // one arrival per softmax warp of the tile
       mbar_init(&o_final[t], 1);
+      mbar_init(&pv_done[t], 1);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -245,35 +252,79 @@ __global__ void __launch_bounds__(576, 1)
       const uint32_t sQ = smem_u32(smem + L::OFF_Q);
       const uint32_t sK = smem_u32(smem + L::OFF_K);
       const uint32_t sV = smem_u32(smem + L::OFF_V);
-      auto issue_S = [&](int t, int st) {
+      // S_t = Q_t K^T into the 128 TMEM columns at `buf`.
+      auto issue_S = [&](int t, int st, uint32_t buf) {
         const uint64_t qd = desc_sw128(sQ + t * L::TILE, 16, 1024);
         const uint64_t kd = desc_sw128(sK + st * L::TILE, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {  // 32 bytes of the head dim per instruction
           const uint32_t o = (kk >> 2) * L::BLK + (kk & 3) * 32;
-          mma_ss_w(tmem + t * 128, desc_add(qd, o), desc_add(kd, o), idS, kk > 0);
+          mma_ss_w(tmem + buf, desc_add(qd, o), desc_add(kd, o), idS, kk > 0);
         }
       };
-      auto issue_PV = [&](int t, int st, int acc) {
+      // O_t += P_t V with P_t over the S buffer at `buf`.
+      auto issue_PV = [&](int t, int st, uint32_t buf, int acc) {
         const uint64_t vd = desc_sw128(sV + st * L::TILE, L::BLK, 1024);
-        // Keys 16kk .. 16kk + 15: P of half kk >> 2 at columns 128t + 64(kk >> 2)
+        // Keys 16kk .. 16kk + 15: P of half kk >> 2 at columns buf + 64(kk >> 2)
         // + 8(kk & 3) (8 columns per 16 keys); V advances 16 rows of 128 bytes.
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts_w(tmem + 256 + t * D, tmem + t * 128 + 64 * (kk >> 2) + (kk & 3) * 8, desc_add(vd, kk * 2048), idO,
+          mma_ts_w(tmem + OBASE + t * D, tmem + buf + 64 * (kk >> 2) + (kk & 3) * 8, desc_add(vd, kk * 2048), idO,
                    (acc || kk > 0) ? 1u : 0u);
       };
-      bool ok = wait(q_full, 0, -1) && wait(&k_full[0], 0, 0);
-      if (ok) {
+      bool ok = wait(q_full, 0, -1);
+      if constexpr (kRot3) {
+        // S products in the order k = 2j + t (block j, tile t), the k-th into
+        // buffer k % 3; P_t(j) overwrites its S there. S(k + 3) is issued
+        // right after P V(k), the last reader of the buffer it reuses (the
+        // tensor core runs them in issue order), so every S is ready well
+        // before the softmax warps reach it. s_full[t] completes once per
+        // block of tile t, pv_done[t] once per P_t(j) V_j.
+        int kwait = -1, vwait = -1;  // last block whose K / V arrival was awaited
+        auto s_exists = [&](int k) { return (k >> 1) < ((k & 1) ? nkv[1] : nkv[0]); };
+        auto issue_S_k = [&](int k) {
+          const int t = k & 1, j = k >> 1;
+          if (j > kwait) {
+            if (!wait(&k_full[j % S], (j / S) & 1, j)) return false;
+            tc_fence_after();
+            kwait = j;
+          }
+          issue_S(t, j % S, 128 * (k % 3));
+          mma_commit_w(&s_full[t]);
+          // K_j is free after its last S (tile 1's, or tile 0's where tile 1
+          // has no block j).
+          if (t == 1 || j >= nkv[1]) mma_commit_w(&k_empty[j % S]);
+          return true;
+        };
+        for (int k = 0; ok && k < 3; ++k)
+          if (s_exists(k)) ok = issue_S_k(k);
+        for (int k = 0; ok && k < 2 * nmax; ++k) {
+          const int t = k & 1, j = k >> 1;
+          const int nt = t ? nkv[1] : nkv[0];
+          if (j < nt) {
+            if (j > vwait) {
+              if (!(ok = wait(&v_full[j % S], (j / S) & 1, j))) break;
+              vwait = j;
+            }
+            if (!(ok = wait(&p_full[t], j & 1, j))) break;
+            tc_fence_after();
+            issue_PV(t, j % S, 128 * (k % 3), j > 0);
+            mma_commit_w(&pv_done[t]);
+            if (j == nt - 1) mma_commit_w(&o_final[t]);
+            if (t == 1 || j >= nkv[1]) mma_commit_w(&v_empty[j % S]);
+          }
+          if (s_exists(k + 3)) ok = issue_S_k(k + 3);
+        }
+      } else if (ok && (ok = wait(&k_full[0], 0, 0))) {
         tc_fence_after();
         for (int t = 0; t < 2; ++t)
           if (nkv[t] > 0) {
-            issue_S(t, 0);
+            issue_S(t, 0, 128 * t);
             mma_commit_w(&s_full[t]);
           }
         mma_commit_w(&k_empty[0]);
       }
-      for (int j = 0; ok && j < nmax; ++j) {
+      for (int j = 0; ok && !kRot3 && j < nmax; ++j) {
         const int st = j % S;
         const uint32_t ph = (j / S) & 1;
         const int jn = j + 1;
@@ -287,7 +338,7 @@ __global__ void __launch_bounds__(576, 1)
           if (j < nkv[t]) {
             if (!(ok = wait(&p_full[t], j & 1, j))) break;
             tc_fence_after();
-            issue_PV(t, st, j > 0);
+            issue_PV(t, st, 128 * t, j > 0);
             if (j == nkv[t] - 1) mma_commit_w(&o_final[t]);
             // V_j is free once the last P V that reads it has run (tile 1's,
             // or tile 0's where tile 1 has no block j): the loader may refill
@@ -300,7 +351,7 @@ __global__ void __launch_bounds__(576, 1)
               tc_fence_after();
               kn_ready = true;
             }
-            issue_S(t, stn);
+            issue_S(t, stn, 128 * t);
             mma_commit_w(&s_full[t]);
           }
         }
@@ -321,8 +372,7 @@ __global__ void __launch_bounds__(576, 1)
     const int n = t ? nkv[1] : nkv[0];
     const int pair_bar = 1 + t * 4 + quarter;  // named barrier of the two warps that share these rows
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t tS = tmem + lane_base + t * 128 + 64 * c;          // this half's S, then its P
-    const uint32_t tO = tmem + lane_base + 256 + t * D + c * (D / 2);  // this half's O columns
+    const uint32_t tO = tmem + lane_base + OBASE + t * D + c * (D / 2);  // this half's O columns
     const float sl2 = a.scale_log2;
     const int off = a.Sk - a.Sq;
     float m = -INFINITY;  // running max of x = s * scale * log2(e), the same in both halves
@@ -330,12 +380,16 @@ __global__ void __launch_bounds__(576, 1)
     bool ok = true;
 
     for (int j = 0; j < n; ++j) {
-      const bool ready = __all_sync(0xffffffffu, wait_bar(&s_full[t], j & 1, abort_flag, kRoleSoftmax, j));
+      // `ok` false here: a wait of the previous block ran out; this warp goes
+      // straight to the pair barrier, which then ends both warps.
+      const bool ready = ok && __all_sync(0xffffffffu, wait_bar(&s_full[t], j & 1, abort_flag, kRoleSoftmax, j));
       const int k0 = j * 128 + 64 * c;  // first key of this half
       const bool masked = k0 + 64 > a.Sk || (a.causal && k0 + 63 > r0 + off);
       int lim = a.Sk - 1 - k0;  // last allowed column of this half
       if (a.causal) lim = min(lim, row + off - k0);
       float* slot = pmax + (((j & 1) * 2 + t) * 2) * 128;
+      // This half's S of block j, then its P (D = 64: buffer (2j + t) % 3).
+      const uint32_t tS = tmem + lane_base + 128 * (kRot3 ? (2 * j + t) % 3 : t) + 64 * c;
       float pm = -INFINITY;
       if (ready) {
         tc_fence_after();
@@ -345,26 +399,25 @@ __global__ void __launch_bounds__(576, 1)
         tmem_ld_wait();
         reg_fence(rr[0]);
         reg_fence(rr[1]);
-        float x[64];
-#pragma unroll
-        for (int q = 0; q < 2; ++q)
-#pragma unroll
-          for (int i = 0; i < 32; ++i) x[32 * q + i] = __uint_as_float(rr[q][i]);
         if (masked) {
 #pragma unroll
-          for (int i = 0; i < 64; ++i) x[i] = (i <= lim) ? x[i] : -INFINITY;
+          for (int q = 0; q < 2; ++q)
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              rr[q][i] = (32 * q + i <= lim) ? rr[q][i] : __float_as_uint(-INFINITY);
         }
-        float mx0 = max3(x[0], x[1], x[2]), mx1 = max3(x[3], x[4], x[5]);
-        float mx2 = max3(x[6], x[7], x[8]), mx3 = max3(x[9], x[10], x[11]);
+        auto xf = [&](int i) { return __uint_as_float(rr[i >> 5][i & 31]); };
+        float mx0 = max3(xf(0), xf(1), xf(2)), mx1 = max3(xf(3), xf(4), xf(5));
+        float mx2 = max3(xf(6), xf(7), xf(8)), mx3 = max3(xf(9), xf(10), xf(11));
 #pragma unroll
         for (int i = 12; i < 60; i += 8) {
-          mx0 = max3(mx0, x[i], x[i + 1]);
-          mx1 = max3(mx1, x[i + 2], x[i + 3]);
-          mx2 = max3(mx2, x[i + 4], x[i + 5]);
-          mx3 = max3(mx3, x[i + 6], x[i + 7]);
+          mx0 = max3(mx0, xf(i), xf(i + 1));
+          mx1 = max3(mx1, xf(i + 2), xf(i + 3));
+          mx2 = max3(mx2, xf(i + 4), xf(i + 5));
+          mx3 = max3(mx3, xf(i + 6), xf(i + 7));
         }
-        mx0 = max3(mx0, x[60], x[61]);
-        mx1 = max3(mx1, x[62], x[63]);
+        mx0 = max3(mx0, xf(60), xf(61));
+        mx1 = max3(mx1, xf(62), xf(63));
         pm = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
         // The slot of block j is written again in block j + 2, after the
         // partner has passed the barrier of block j + 1, i.e. after it has
@@ -385,10 +438,17 @@ __global__ void __launch_bounds__(576, 1)
         m = m_blk;
       }
       l *= alpha;
-      if (j > 0 && __any_sync(0xffffffffu, raise)) {
+      // P_t(j-1) V_{j-1} must have completed before O_t is rescaled. D = 128:
+      // S_t(j) was issued after it and s_full covers both. D = 64: S_t(j) may
+      // have been issued before it, so wait for pv_done.
+      const bool rescale = j > 0 && __any_sync(0xffffffffu, raise);
+      if (kRot3 && rescale &&
+          !__all_sync(0xffffffffu, wait_bar(&pv_done[t], (j - 1) & 1, abort_flag, kRoleSoftmax, j))) {
+        ok = false;  // the next pair barrier (or the epilogue's) ends both warps
+        continue;
+      }
+      if (rescale) {
         // Rescale this warp's 32 rows of this half's D/2 columns of O_t.
-        // P V(j-1) has completed: S(j) was issued after it and s_full(j)
-        // covers both.
 #pragma unroll 1
         for (int q = 0; q < D / 64; ++q) {
           uint32_t ov[32];
@@ -436,9 +496,9 @@ __global__ void __launch_bounds__(576, 1)
     // Epilogue: O = O_t / (l_0 + l_1), LSE = ln2 * (m + log2(l_0 + l_1)).
     // Both warps of the pair arrive here with the same `ok` (the loop's
     // barrier ANDs it), so both take the barrier below or neither does.
-    if (ok && r0 < a.Sq) {
+    if (r0 < a.Sq) {
       lsum[(t * 2 + c) * 128 + r] = l;
-      const bool go = named_bar_and(pair_bar, 64, !*abort_flag);
+      const bool go = named_bar_and(pair_bar, 64, ok && !*abort_flag);
       const bool valid = row < a.Sq;
       const int cb = c * (D / 2);  // first O column of this half
       uint16_t* orow = reinterpret_cast<uint16_t*>(a.o) + static_cast<int64_t>(b) * a.o_sb +
