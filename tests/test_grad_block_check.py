@@ -45,6 +45,20 @@ def test_block_check_catches_one_missing_block_pair():
     check_grad(dk, dk, "unperturbed", row_axis=1, head_axes=(0, 2))
 
 
+def test_sampled_rows_are_checked_per_head():
+    rng = np.random.default_rng(5)
+    ref = rng.standard_normal((3, 40, 8))
+    got = ref.copy()
+    # one sampled row off by 7% of its head's norm: 4% of the whole tensor
+    got[1, 7] += 0.07 * np.linalg.norm(ref[1]) / np.sqrt(ref.shape[2])
+    check_grad(got, ref, "whole tensor only")
+    with pytest.raises(AssertionError, match="head index \\(1,\\)"):
+        check_grad(got, ref, "sampled", row_axis=1, head_axes=(0,), rows="sampled")
+    got = ref.copy()
+    got[1, 7] += 0.03 * np.linalg.norm(ref[1]) / np.sqrt(ref.shape[2])
+    check_grad(got, ref, "sampled", row_axis=1, head_axes=(0,), rows="sampled")
+
+
 def test_block_check_groups_sampled_rows_and_floors_near_zero_pieces():
     rng = np.random.default_rng(3)
     ref = rng.standard_normal((2, 40, 8))
