@@ -89,14 +89,37 @@ int make_map(CUtensorMap* map, const fa_tensor& t, int B, int S, int H, int D, i
   return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
 
-// Raises the dynamic shared memory limit of `fn` once per device.
+// 2-D map over the fp32 dQ accumulator [rows][64], boxes of 32 rows x 32
+// floats (128 bytes) in the 128-byte swizzled shared-memory layout: the D = 64
+// backward stages dQ blocks that way and has the TMA add them.
+int make_dq_map(CUtensorMap* map, float* acc, int64_t rows) {
+  auto fn = encode_fn();
+  if (!fn) return FA_ERR_CUDA;
+  cuuint64_t dims[2] = {64, cuuint64_t(rows)};
+  cuuint64_t strides[1] = {64 * sizeof(float)};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, acc, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
+// Raises the dynamic shared memory limit of `fn` once per device, and asks
+// for the largest shared-memory carveout. Every kernel of the library asks
+// for the same carveout, so consecutive launches (forward, backward
+// preprocess, main, dQ convert) never make the SM reconfigure its L1/shared
+// split between them.
 template <typename F>
 int prepare(F* fn, int smem_bytes, bool (&done)[kMaxDevices]) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
   if (!done[dev]) {
-    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) != cudaSuccess)
+    if (smem_bytes > 0 &&
+        cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) != cudaSuccess)
+      return FA_ERR_CUDA;
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared) !=
+        cudaSuccess)
       return FA_ERR_CUDA;
     done[dev] = true;
   }
@@ -220,11 +243,19 @@ int launch_bwd(const fa_bwd_params* p, cudaStream_t stream) {
   a.causal = p->causal;
   a.d = p->D;
   constexpr int G = D / 8;
+  {
+    static bool done_pre[kMaxDevices] = {}, done_dq[kMaxDevices] = {}, done_sum[kMaxDevices] = {};
+    if ((st = prepare(&fa::fa_bwd_pre<D, BF16>, 0, done_pre)) != FA_OK) return st;
+    if ((st = prepare(&fa::fa_bwd_dq<D, BF16>, 0, done_dq)) != FA_OK) return st;
+    if ((st = prepare(&fa::fa_bwd_dq_sum<D, BF16>, 0, done_sum)) != FA_OK) return st;
+  }
   const int64_t pre_threads = rows * G;
   fa::fa_bwd_pre<D, BF16><<<unsigned((pre_threads + 255) / 256), 256, 0, stream>>>(a);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   const unsigned grid = unsigned(int64_t((p->Sk + L::BN - 1) / L::BN) * p->B * p->H);
-  kern<<<grid, L::kThreads, L::SMEM_ALLOC, stream>>>(mq, mk, mv, mdo, a);
+  CUtensorMap mdq = mq;  // D = 128 does not read it
+  if (D == 64 && (st = make_dq_map(&mdq, a.dq_acc, rows)) != FA_OK) return st;
+  kern<<<grid, L::kThreads, L::SMEM_ALLOC, stream>>>(mq, mk, mv, mdo, mdq, a);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   const int64_t dq_threads = int64_t(p->B) * p->H * p->Sq * G;
   if (a.dq_part != nullptr)

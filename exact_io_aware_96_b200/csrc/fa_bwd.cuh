@@ -178,7 +178,7 @@ struct BwdLayout {
   static constexpr int BM = 128;         // query rows per block
   // Q (with lse2) and dO (with Dvec) travel on separate rings: S^T(i+1)
   // needs Q(i+1) right after dV(i), dP^T(i+1) needs dO(i+1) later in block
-  // i, after dO(i) has been released, so one dO stage suffices.
+  // i, after dO(i) has been released.
   // Q stages: three where shared memory allows (D = 64); D = 128 spends the
   // third stage's 32 KB on the dQ staging buffers below.
   static constexpr int QS = (D == 128) ? 2 : 3;
@@ -227,7 +227,8 @@ struct BwdLayout {
 template <int D, bool BF16>
 __global__ void __launch_bounds__(448, 1)
     fa_bwd_main(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO, const BwdArgs a) {
+                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                const __grid_constant__ CUtensorMap tmDQ, const BwdArgs a) {
   using L = BwdLayout<D>;
   using namespace sm100;
   constexpr int BM = L::BM, QS = L::QS;
@@ -323,8 +324,9 @@ __global__ void __launch_bounds__(448, 1)
           tma_load_4d(smem + L::OFF_K + kb * L::BLK, &tmK, kv_full, kb * 64, n0, h, b);
           tma_load_4d(smem + L::OFF_V + kb * L::BLK, &tmV, kv_full, kb * 64, n0, h, b);
         }
-        // Q(j) with lse2(j) runs QS - 1 blocks ahead of dO(j) with Dvec(j):
-        // per step, dO(i) (its slot frees first) and then Q(i + QS - 1).
+        // Q(j) with lse2(j) runs QS - 1 blocks ahead, dO(j) with Dvec(j)
+        // OS - 1 blocks ahead: per step i, dO(i + OS - 1) (at OS = 1 its slot
+        // frees first) and then Q(i + QS - 1).
         int nq = 0, no = 0;  // loads issued
         auto load_q = [&](int j) -> bool {
           const int st = j % QS;
@@ -350,8 +352,9 @@ __global__ void __launch_bounds__(448, 1)
         };
         bool lok = true;
         for (int j = 0; lok && j < QS - 1 && j < n; ++j) lok = load_q(j);
+        for (int j = 0; lok && j < L::OS - 1 && j < n; ++j) lok = load_o(j);
         for (int i = 0; lok && i < n; ++i) {
-          lok = load_o(i);
+          if (i + L::OS - 1 < n) lok = load_o(i + L::OS - 1);
           if (lok && i + QS - 1 < n) lok = load_q(i + QS - 1);
         }
         if (*abort_flag) {
@@ -734,22 +737,31 @@ __global__ void __launch_bounds__(448, 1)
                     make_float4(__uint_as_float(v[part][c]), __uint_as_float(v[part][c + 1]),
                                 __uint_as_float(v[part][c + 2]), __uint_as_float(v[part][c + 3]));
           } else {
-            // This warp's 32 rows are contiguous in the accumulator: stage
-            // them as rows of D floats and let the TMA add the 8 KB.
+            // This warp's 32 rows are contiguous in the accumulator. They are
+            // staged as two boxes of 32 rows x 32 floats (columns 0-31 and
+            // 32-63) in the 128-byte swizzled layout: row r's 16-byte chunk c
+            // sits at r * 128 + ((c ^ (r % 8)) * 16), so the eight lanes of
+            // each store phase hit eight different bank groups (rows of 256
+            // plain bytes would put all 32 lanes on the same banks). The TMA
+            // reads the swizzle through tmDQ and adds each box into the
+            // accumulator.
             const int wq = warp & 3;
             uint8_t* wbuf = smem + L::OFF_DQS + wq * L::DQ_PART;
             if (lane == 0) bulk_wait_read0();  // this warp's previous reduction has read the buffer
             __syncwarp();
-            const uint32_t rbuf = smem_u32(wbuf) + lane * (D * 4);
+            const uint32_t rbase = smem_u32(wbuf) + lane * 128;
 #pragma unroll
             for (int part = 0; part < D / 32; ++part)
 #pragma unroll
-              for (int c = 0; c < 32; c += 4)
-                st_shared_v4(rbuf + (32 * part + c) * 4, v[part][c], v[part][c + 1], v[part][c + 2], v[part][c + 3]);
+              for (int c = 0; c < 8; ++c)
+                st_shared_v4(rbase + part * (32 * 128) + ((c ^ (lane & 7)) << 4), v[part][4 * c],
+                             v[part][4 * c + 1], v[part][4 * c + 2], v[part][4 * c + 3]);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-              bulk_reduce_add_f32(base + (32 * wq) * D, wbuf, L::DQ_PART);
+              const int row0 = static_cast<int>(bh_row0 + static_cast<int64_t>(qb) * BM) + 32 * wq;
+#pragma unroll
+              for (int part = 0; part < D / 32; ++part) tma_reduce_add_2d(&tmDQ, wbuf + part * (32 * 128), 32 * part, row0);
               bulk_commit();
             }
           }

@@ -178,6 +178,16 @@ __device__ __forceinline__ void bulk_reduce_add_f32(float* dst, const void* src,
                "r"(smem_u32(src)), "r"(bytes)
                : "memory");
 }
+// Tensor-map form: element-wise fp32 add of a shared-memory box (laid out as
+// the tensor map says, e.g. 128-byte swizzled) into the tile of global memory
+// at coordinates (c0, c1), innermost first; tracked as one bulk group.
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* map, const void* src, int c0, int c1) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(smem_u32(src)), "r"(c0), "r"(c1)
+      : "memory");
+}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Wait until the source reads of every committed bulk group have finished.
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
