@@ -27,9 +27,15 @@ def nvcc() -> str:
     raise RuntimeError("nvcc not found")
 
 
-def build(verbose: bool = False, extra: list[str] | None = None) -> str:
+LIB_CHECK = os.path.join(HERE, "libfa_check.so")
+
+
+def build(verbose: bool = False, extra: list[str] | None = None, check: bool = False) -> str:
+    """Build libfa.so, or with check=True libfa_check.so: the same sources
+    compiled with FA_CHECK=1 (device-side index and bounds checks)."""
+    out = LIB_CHECK if check else LIB
     cmd = [nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2", "-shared",
-           "-I" + INCLUDE, "-I" + CSRC, "-o", LIB + ".tmp", *SOURCES]
+           "-I" + INCLUDE, "-I" + CSRC, "-o", out + ".tmp", *(["-DFA_CHECK=1"] if check else []), *SOURCES]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     if extra:
@@ -37,11 +43,11 @@ def build(verbose: bool = False, extra: list[str] | None = None) -> str:
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         raise RuntimeError("nvcc failed:\n" + res.stdout + res.stderr)
-    os.replace(LIB + ".tmp", LIB)
+    os.replace(out + ".tmp", out)
     if verbose:
         sys.stdout.write(res.stdout + res.stderr)
-    return LIB
+    return out
 
 
 if __name__ == "__main__":
-    print(build(verbose="-v" in sys.argv))
+    print(build(verbose="-v" in sys.argv, check="--check" in sys.argv))

@@ -311,6 +311,7 @@ const char* fa_strerror(int s) {
     case FA_ERR_NOT_IMPLEMENTED: return "not implemented";
     case FA_ERR_WORKSPACE: return "workspace missing or smaller than fa_bwd_workspace_size()";
     case FA_ERR_SCRATCH_LIMIT: return "fa_bwd_noalloc: the problem needs more scratch than FA_NOALLOC_SCRATCH_BYTES (64 MiB)";
+    case FA_ERR_BOUNDS: return "a device-side index or bounds check failed (check build); the access was skipped";
     default: return "unknown status";
   }
 }

@@ -74,7 +74,7 @@ __global__ void __launch_bounds__(256) fa_bwd_pre(const BwdArgs a) {
   const int h = bh % a.H;
   const int b = bh / a.H;
   float acc = 0.f;
-  if (i < a.Sq && part * 8 < a.d) {
+  if (i < a.Sq && part * 8 < a.d && checked(b < a.B && h < a.H && part * 8 + 8 <= D, 201)) {
     const uint4 ov = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(a.o) + b * a.o_sb +
                                                       static_cast<int64_t>(i) * a.o_ss + h * a.o_sh + part * 8);
     const uint4 dv = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(a.dO) + b * a.do_sb +
@@ -91,12 +91,12 @@ __global__ void __launch_bounds__(256) fa_bwd_pre(const BwdArgs a) {
   }
 #pragma unroll
   for (int s = G / 2; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
-  if (a.dq_part == nullptr) {  // the atomic accumulator starts from zero
+  if (a.dq_part == nullptr && checked(row < nrows && part * 8 + 8 <= D, 202)) {  // the atomic accumulator starts from zero
     float4* dq = reinterpret_cast<float4*>(a.dq_acc + row * D + part * 8);
     dq[0] = make_float4(0.f, 0.f, 0.f, 0.f);
     dq[1] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  if (part == 0) {
+  if (part == 0 && checked(row < nrows, 203)) {
     a.dvec[row] = acc;
     float l2 = INFINITY;
     if (i < a.Sq) {
@@ -119,6 +119,7 @@ __global__ void __launch_bounds__(256) fa_bwd_dq(const BwdArgs a) {
   const int bh = static_cast<int>(row / a.Sq);
   const int h = bh % a.H;
   const int b = bh / a.H;
+  if (!checked(b < a.B && i < a.Sq_pad && part * 8 + 8 <= D, 206)) return;
   const float4* src = reinterpret_cast<const float4*>(a.dq_acc + (static_cast<int64_t>(bh) * a.Sq_pad + i) * D +
                                                       part * 8);
   const float4 x = src[0], y = src[1];
@@ -150,6 +151,7 @@ __global__ void __launch_bounds__(256) fa_bwd_dq_sum(const BwdArgs a) {
   const int h = bh % a.H;
   const int b = bh / a.H;
   const int qb = i / 128;
+  if (!checked(b < a.B && qb < a.nqb && part * 8 + 8 <= D, 207)) return;
   const float* slot = a.dq_part + (static_cast<int64_t>(bh) * a.nqb + qb) * a.nkb * (128 * D) +
                       (i % 128) * D + part * 8;
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -320,6 +322,9 @@ __global__ void __launch_bounds__(448, 1)
       // ---------------------------------------------------------------- loader
       if (lane == 0 && n > 0) {
         mbar_arrive_expect_tx(kv_full, 2 * L::TILE);
+        // TMA zero-fills tiles past the tensor's end; the check build still
+        // records a tile that starts outside it (a scheduling error).
+        checked(n0 < a.Sk && b < a.B && h < a.H, 210);
         for (int kb = 0; kb < L::KB; ++kb) {
           tma_load_4d(smem + L::OFF_K + kb * L::BLK, &tmK, kv_full, kb * 64, n0, h, b);
           tma_load_4d(smem + L::OFF_V + kb * L::BLK, &tmV, kv_full, kb * 64, n0, h, b);
@@ -332,10 +337,13 @@ __global__ void __launch_bounds__(448, 1)
           const int st = j % QS;
           if (!wait_bar(&q_empty[st], ((j / QS) & 1) ^ 1, abort_flag, kRoleLoader, j)) return false;
           const int j0 = (i_start + j) * BM;
+          checked(j0 < a.Sq, 211);
           mbar_arrive_expect_tx(&q_full[st], L::TILE + BM * 4);
           for (int kb = 0; kb < L::KB; ++kb)
             tma_load_4d(smem + L::OFF_Q + st * L::TILE + kb * L::BLK, &tmQ, &q_full[st], kb * 64, j0, h, b);
-          bulk_load(smem + L::OFF_LSE + st * BM * 4, a.lse2 + bh_row0 + j0, BM * 4, &q_full[st]);
+          // Skipped on a failed check: its wait then runs out (FA_ERR_BOUNDS stays recorded).
+          if (checked(bh_row0 + j0 + BM <= static_cast<int64_t>(a.B) * a.H * a.Sq_pad, 212))
+            bulk_load(smem + L::OFF_LSE + st * BM * 4, a.lse2 + bh_row0 + j0, BM * 4, &q_full[st]);
           ++nq;
           return true;
         };
@@ -343,10 +351,12 @@ __global__ void __launch_bounds__(448, 1)
           const int st = j % L::OS;
           if (!wait_bar(&o_empty[st], ((j / L::OS) & 1) ^ 1, abort_flag, kRoleLoader, j)) return false;
           const int j0 = (i_start + j) * BM;
+          checked(j0 < a.Sq, 211);
           mbar_arrive_expect_tx(&o_full[st], L::TILE + BM * 4);
           for (int kb = 0; kb < L::KB; ++kb)
             tma_load_4d(smem + L::OFF_DO + st * L::TILE + kb * L::BLK, &tmdO, &o_full[st], kb * 64, j0, h, b);
-          bulk_load(smem + L::OFF_DVEC + st * BM * 4, a.dvec + bh_row0 + j0, BM * 4, &o_full[st]);
+          if (checked(bh_row0 + j0 + BM <= static_cast<int64_t>(a.B) * a.H * a.Sq_pad, 212))
+            bulk_load(smem + L::OFF_DVEC + st * BM * 4, a.dvec + bh_row0 + j0, BM * 4, &o_full[st]);
           ++no;
           return true;
         };
@@ -622,7 +632,7 @@ __global__ void __launch_bounds__(448, 1)
               for (int e = 0; e < 4; ++e)
                 w[e] = pack2<BF16>(__uint_as_float(v[8 * u + 2 * e]) * mul,
                                    __uint_as_float(v[8 * u + 2 * e + 1]) * mul);
-              if (32 * c + 8 * u < a.d) d4[u] = make_uint4(w[0], w[1], w[2], w[3]);
+              if (32 * c + 8 * u < a.d && checked(b < a.B && h < a.H, 217)) d4[u] = make_uint4(w[0], w[1], w[2], w[3]);
             }
           }
         }
@@ -636,7 +646,9 @@ __global__ void __launch_bounds__(448, 1)
     // adding it into the shared accumulator.
     auto drain = [&](auto det) {
       constexpr bool DET = decltype(det)::value;
+      bool in_range = true;  // set per block below
       auto put = [&](float* p, float x) {
+        if (!in_range) return;
         if constexpr (DET)
           *p = x;
         else
@@ -653,6 +665,11 @@ __global__ void __launch_bounds__(448, 1)
         // block base: row0 of the accumulator, or the (qb, kvb) slot
         float* base = DET ? a.dq_part + ((static_cast<int64_t>(hb) * a.nqb + qb) * a.nkb + kvb) * (BM * D)
                           : a.dq_acc + (bh_row0 + static_cast<int64_t>(qb) * BM) * D;
+        // Every write of this block lands in [base, base + BM * D); the check
+        // build skips the block if that range leaves its buffer.
+        in_range =
+            DET ? checked(hb < a.B * a.H && qb < a.nqb && kvb < a.nkb, 216)
+                : checked(bh_row0 + static_cast<int64_t>(qb) * BM + BM <= static_cast<int64_t>(a.B) * a.H * a.Sq_pad, 216);
         if constexpr (L::DQ_T) {
           // lane = head_dim index d, columns = 128 query rows: for each query the
           // warp writes 32 consecutive floats (one 128-byte line). Three quarters
@@ -698,7 +715,10 @@ __global__ void __launch_bounds__(448, 1)
             auto reduce = [&](int part) {
               named_bar_sync(1, 128);
               if (warp == 8 && lane == 0) {
-                bulk_reduce_add_f32(base + 32 * part * D, smem + L::OFF_DQS + (part & 1) * L::DQ_PART, L::DQ_PART);
+                if (checked(bh_row0 + static_cast<int64_t>(qb) * BM + 32 * part + 32 <=
+                                static_cast<int64_t>(a.B) * a.H * a.Sq_pad,
+                            214))
+                  bulk_reduce_add_f32(base + 32 * part * D, smem + L::OFF_DQS + (part & 1) * L::DQ_PART, L::DQ_PART);
                 bulk_commit();
               }
             };
@@ -733,9 +753,10 @@ __global__ void __launch_bounds__(448, 1)
             for (int part = 0; part < D / 32; ++part)
 #pragma unroll
               for (int c = 0; c < 32; c += 4)
-                *reinterpret_cast<float4*>(row + 32 * part + c) =
-                    make_float4(__uint_as_float(v[part][c]), __uint_as_float(v[part][c + 1]),
-                                __uint_as_float(v[part][c + 2]), __uint_as_float(v[part][c + 3]));
+                if (in_range)
+                  *reinterpret_cast<float4*>(row + 32 * part + c) =
+                      make_float4(__uint_as_float(v[part][c]), __uint_as_float(v[part][c + 1]),
+                                  __uint_as_float(v[part][c + 2]), __uint_as_float(v[part][c + 3]));
           } else {
             // This warp's 32 rows are contiguous in the accumulator. They are
             // staged as two boxes of 32 rows x 32 floats (columns 0-31 and
@@ -761,7 +782,9 @@ __global__ void __launch_bounds__(448, 1)
             if (lane == 0) {
               const int row0 = static_cast<int>(bh_row0 + static_cast<int64_t>(qb) * BM) + 32 * wq;
 #pragma unroll
-              for (int part = 0; part < D / 32; ++part) tma_reduce_add_2d(&tmDQ, wbuf + part * (32 * 128), 32 * part, row0);
+              if (checked(row0 + 32 <= static_cast<int64_t>(a.B) * a.H * a.Sq_pad, 215))
+                for (int part = 0; part < D / 32; ++part)
+                  tma_reduce_add_2d(&tmDQ, wbuf + part * (32 * 128), 32 * part, row0);
               bulk_commit();
             }
           }

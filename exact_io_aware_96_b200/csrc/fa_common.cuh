@@ -17,7 +17,30 @@ namespace fa {
 // its own copy of a __device__ variable).
 __device__ int g_status[4];
 
-enum Role : int { kRoleLoader = 1, kRoleMma = 2, kRoleSoftmax = 3, kRoleSelfTest = 4 };
+enum Role : int { kRoleLoader = 1, kRoleMma = 2, kRoleSoftmax = 3, kRoleSelfTest = 4, kRoleCheck = 5 };
+
+// The check build (-DFA_CHECK=1, libfa_check.so): checked(ok, site) records a
+// failed index or bounds test in the status word (FA_ERR_BOUNDS, role 5, the
+// site number in place of the loop index) and returns false, so that the
+// caller skips the access. In the normal build it is `true` and the test is
+// not compiled. Sites: 1xx 16-bit forward, 2xx backward, 3xx e4m3 forward.
+#ifndef FA_CHECK
+#define FA_CHECK 0
+#endif
+__device__ __forceinline__ bool checked(bool ok, int site) {
+#if FA_CHECK
+  if (!ok && atomicCAS(&g_status[0], 0, -9) == 0) {
+    g_status[1] = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
+    g_status[2] = kRoleCheck;
+    g_status[3] = site;
+  }
+  return ok;
+#else
+  (void)ok;
+  (void)site;
+  return true;
+#endif
+}
 
 // A wait longer than this is treated as a hang: the kernel records it and
 // winds down instead of spinning forever. Real waits last microseconds.

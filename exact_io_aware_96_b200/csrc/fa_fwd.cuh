@@ -155,15 +155,18 @@ __global__ void __launch_bounds__(320, 1)
       for (int t = 0; t < 2; ++t) q_bytes += nkv[t] > 0 ? L::TILE : 0;
       mbar_arrive_expect_tx(q_full, q_bytes);
       for (int t = 0; t < 2; ++t)
-        if (nkv[t] > 0)
+        if (nkv[t] > 0) {
+          checked(q0 + 128 * t < a.Sq && b < a.B && h < a.H, 301);
           for (int kb = 0; kb < L::KB; ++kb)
             tma_load_4d(smem + L::OFF_Q + t * L::TILE + kb * L::BLK, &tmQ, q_full, kb * KCOL, q0 + 128 * t, h, b);
+        }
       int j = 0;
       for (; j < nmax; ++j) {
         const int st = j % S;
         const uint32_t ph = (j / S) & 1;
         if (!wait_bar(&k_empty[st], ph ^ 1, abort_flag, kRoleLoader, j)) break;
         mbar_arrive_expect_tx(&k_full[st], L::TILE);
+        checked(j * 128 < a.Sk && st < S, 302);
         for (int kb = 0; kb < L::KB; ++kb)
           tma_load_4d(smem + L::OFF_K + st * L::TILE + kb * L::BLK, &tmK, &k_full[st], kb * KCOL, j * 128, h, b);
         if (!wait_bar(&v_empty[st], ph ^ 1, abort_flag, kRoleLoader, j)) {
@@ -415,15 +418,17 @@ __global__ void __launch_bounds__(320, 1)
               uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
 #pragma unroll
               for (int i = 0; i < 4; ++i)
-                if (32 * c + 8 * i < a.d) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                if (32 * c + 8 * i < a.d && checked(row < a.Sq && b < a.B && h < a.H, 307))
+                  dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
             }
           }
         }
       } else if (valid) {
         uint4* dst = reinterpret_cast<uint4*>(orow);
-        for (int i = 0; i < a.d / 8; ++i) dst[i] = make_uint4(0, 0, 0, 0);
+        if (checked(row < a.Sq && b < a.B && h < a.H, 309))
+          for (int i = 0; i < a.d / 8; ++i) dst[i] = make_uint4(0, 0, 0, 0);
       }
-      if (valid)
+      if (valid && checked(b < a.B && h < a.H && row < a.Sq, 308))
         a.lse[(static_cast<int64_t>(b) * a.H + h) * a.Sq + row] =
             has ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
     }

@@ -210,15 +210,20 @@ __global__ void __launch_bounds__(576, 1)
       for (int t = 0; t < 2; ++t) q_bytes += nkv[t] > 0 ? L::TILE : 0;
       mbar_arrive_expect_tx(q_full, q_bytes);
       for (int t = 0; t < 2; ++t)
-        if (nkv[t] > 0)
+        if (nkv[t] > 0) {
+          // TMA zero-fills tiles past the tensor's end; the check build still
+          // records a tile that starts outside it (a scheduling error).
+          checked(q0 + 128 * t < a.Sq && b < a.B && h < a.H, 101);
           for (int kb = 0; kb < L::KB; ++kb)
             tma_load_4d(smem + L::OFF_Q + t * L::TILE + kb * L::BLK, &tmQ, q_full, kb * 64, q0 + 128 * t, h, b);
+        }
       int j = 0;
       for (; j < nmax; ++j) {
         const int st = j % S;
         const uint32_t ph = (j / S) & 1;
         if (!wait_bar(&k_empty[st], ph ^ 1, abort_flag, kRoleLoader, j)) break;
         mbar_arrive_expect_tx(&k_full[st], L::TILE);
+        checked(j * 128 < a.Sk && st < S, 102);
         for (int kb = 0; kb < L::KB; ++kb)
           tma_load_4d(smem + L::OFF_K + st * L::TILE + kb * L::BLK, &tmK, &k_full[st], kb * 64, j * 128, h, b);
         if (!wait_bar(&v_empty[st], ph ^ 1, abort_flag, kRoleLoader, j)) {
@@ -226,6 +231,7 @@ __global__ void __launch_bounds__(576, 1)
           break;
         }
         mbar_arrive_expect_tx(&v_full[st], L::TILE);
+        checked(j * 128 < a.Sk && st < S, 102);
         for (int kb = 0; kb < L::KB; ++kb)
           tma_load_4d(smem + L::OFF_V + st * L::TILE + kb * L::BLK, &tmV, &v_full[st], kb * 64, j * 128, h, b);
       }
@@ -254,6 +260,7 @@ __global__ void __launch_bounds__(576, 1)
       const uint32_t sV = smem_u32(smem + L::OFF_V);
       // S_t = Q_t K^T into the 128 TMEM columns at `buf`.
       auto issue_S = [&](int t, int st, uint32_t buf) {
+        checked(buf + 128 <= OBASE && st < S && t < 2, 103);
         const uint64_t qd = desc_sw128(sQ + t * L::TILE, 16, 1024);
         const uint64_t kd = desc_sw128(sK + st * L::TILE, 16, 1024);
 #pragma unroll
@@ -264,6 +271,7 @@ __global__ void __launch_bounds__(576, 1)
       };
       // O_t += P_t V with P_t over the S buffer at `buf`.
       auto issue_PV = [&](int t, int st, uint32_t buf, int acc) {
+        checked(buf + 128 <= OBASE && OBASE + (t + 1) * D <= L::TMEM_COLS && st < S, 104);
         const uint64_t vd = desc_sw128(sV + st * L::TILE, L::BLK, 1024);
         // Keys 16kk .. 16kk + 15: P of half kk >> 2 at columns buf + 64(kk >> 2)
         // + 8(kk & 3) (8 columns per 16 keys); V advances 16 rows of 128 bytes.
@@ -390,6 +398,8 @@ __global__ void __launch_bounds__(576, 1)
       float* slot = pmax + (((j & 1) * 2 + t) * 2) * 128;
       // This half's S of block j, then its P (D = 64: buffer (2j + t) % 3).
       const uint32_t tS = tmem + lane_base + 128 * (kRot3 ? (2 * j + t) % 3 : t) + 64 * c;
+      checked(128 * (kRot3 ? (2 * j + t) % 3 : t) + 64 * c + 64 <= OBASE && (((j & 1) * 2 + t) * 2 + 2) * 128 <= 1024,
+              105);
       float pm = -INFINITY;
       if (ready) {
         tc_fence_after();
@@ -523,19 +533,21 @@ __global__ void __launch_bounds__(576, 1)
               uint4* dst = reinterpret_cast<uint4*>(orow + cb + 32 * q);
 #pragma unroll
               for (int i = 0; i < 4; ++i)
-                if (cb + 32 * q + 8 * i < a.d)
+                if (cb + 32 * q + 8 * i < a.d && checked(row < a.Sq && b < a.B && h < a.H, 107))
                   dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
             }
           }
-          if (valid && c == 0)
+          if (valid && c == 0 && checked(b < a.B && h < a.H && row < a.Sq, 108))
             a.lse[(static_cast<int64_t>(b) * a.H + h) * a.Sq + row] =
                 has ? (m + __log2f(lt)) * 0.69314718055994531f : -INFINITY;
         }
       } else if (go && valid) {
         // No key reaches these rows: O = 0, LSE = -inf.
         uint4* dst = reinterpret_cast<uint4*>(orow);
-        for (int i = cb / 8; i < min(a.d, cb + D / 2) / 8; ++i) dst[i] = make_uint4(0, 0, 0, 0);
-        if (c == 0) a.lse[(static_cast<int64_t>(b) * a.H + h) * a.Sq + row] = -INFINITY;
+        if (checked(row < a.Sq && b < a.B && h < a.H, 109)) {
+          for (int i = cb / 8; i < min(a.d, cb + D / 2) / 8; ++i) dst[i] = make_uint4(0, 0, 0, 0);
+          if (c == 0) a.lse[(static_cast<int64_t>(b) * a.H + h) * a.Sq + row] = -INFINITY;
+        }
       }
     }
   }

@@ -16,13 +16,16 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libfa.so")
+# The same library built with device-side index and bounds checks (FA_CHECK=1;
+# see fa_last_device_status in include/fa.h). Selected with use_library().
+LIB_CHECK_PATH = os.path.join(_HERE, "libfa_check.so")
 
 FA_FP16, FA_BF16 = 0, 1
 FA_OK = 0
 STATUS = {
     0: "FA_OK", -1: "FA_ERR_INVALID_ARG", -2: "FA_ERR_UNSUPPORTED", -3: "FA_ERR_MISALIGNED",
     -4: "FA_ERR_CUDA", -5: "FA_ERR_TIMEOUT", -6: "FA_ERR_NOT_IMPLEMENTED", -7: "FA_ERR_WORKSPACE",
-    -8: "FA_ERR_SCRATCH_LIMIT",
+    -8: "FA_ERR_SCRATCH_LIMIT", -9: "FA_ERR_BOUNDS",
 }
 FA_NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 EXPORTED = ("fa_fwd", "fa_fwd_ex", "fa_fwd_fp8", "fa_fwd_fp8_ex", "fa_bwd", "fa_bwd_ex", "fa_bwd_noalloc",
@@ -69,6 +72,15 @@ class FaError(RuntimeError):
 
 
 _lib = None
+
+
+def use_library(path: str) -> None:
+    """Route every call of this module through the library at `path` from now
+    on (LIB_PATH, or LIB_CHECK_PATH for the check build). The library is
+    loaded at the next call."""
+    global _lib, LIB_PATH
+    LIB_PATH = path
+    _lib = None
 
 
 def lib():
@@ -277,6 +289,40 @@ def forward_fp8(q, k, v, q_descale, k_descale, v_descale, causal=False, scale=No
     if st != FA_OK:
         raise FaError(st, "fa_fwd_fp8_ex")
     return out, lse
+
+
+def backward_noalloc(q, k, v, o, lse, do, causal=False, scale=None, dq=None, dk=None, dv=None, stream=None):
+    """dQ, dK, dV through fa_bwd_noalloc: the backward that takes no workspace
+    and uses the library's built-in device scratch (64 MiB per device;
+    larger problems raise with FA_ERR_SCRATCH_LIMIT). The tensors must be
+    dense [B, S, H, D] (the entry point takes no strides). Calls that overlap
+    on the GPU share that scratch and race: see include/fa.h."""
+    B, Sq, H, D, Sk = _dims(q, k)
+    dt = _dtype_code(q)
+    dev = q.device
+    if not q.is_cuda:
+        raise ValueError("tensors must live on a CUDA device (the library has no CPU path)")
+    for name, t, S in (("q", q, Sq), ("k", k, Sk), ("v", v, Sk), ("o", o, Sq), ("do", do, Sq)):
+        _expect(name, t, (B, S, H, D), q.dtype, dev)
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be a dense [B, S, H, D] tensor for fa_bwd_noalloc")
+    _expect_lse(lse, B, H, Sq, dev)
+    if scale is None:
+        scale = D ** -0.5
+    dq = torch.empty((B, Sq, H, D), dtype=q.dtype, device=dev) if dq is None else dq
+    dk = torch.empty((B, Sk, H, D), dtype=q.dtype, device=dev) if dk is None else dk
+    dv = torch.empty((B, Sk, H, D), dtype=q.dtype, device=dev) if dv is None else dv
+    for name, t, S in (("dq", dq, Sq), ("dk", dk, Sk), ("dv", dv, Sk)):
+        _expect(name, t, (B, S, H, D), q.dtype, dev)
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be a dense [B, S, H, D] tensor for fa_bwd_noalloc")
+    with torch.cuda.device(dev):
+        st = fa_bwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
+                            dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, Sq, Sk, D, float(scale),
+                            int(bool(causal)), dt, _stream(stream))
+    if st != FA_OK:
+        raise FaError(st, "fa_bwd_noalloc")
+    return dq, dk, dv
 
 
 def workspace_for(B, H, Sq, D, device, Sk=None, deterministic=False) -> torch.Tensor:

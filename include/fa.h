@@ -85,7 +85,9 @@ typedef enum {
   FA_ERR_TIMEOUT = -5,         /* a device-side pipeline wait ran out (fa_last_device_status) */
   FA_ERR_NOT_IMPLEMENTED = -6, /* reserved */
   FA_ERR_WORKSPACE = -7,       /* workspace pointer null or smaller than fa_bwd_workspace_size */
-  FA_ERR_SCRATCH_LIMIT = -8    /* fa_bwd_noalloc: problem needs more than FA_NOALLOC_SCRATCH_BYTES */
+  FA_ERR_SCRATCH_LIMIT = -8,   /* fa_bwd_noalloc: problem needs more than FA_NOALLOC_SCRATCH_BYTES */
+  FA_ERR_BOUNDS = -9           /* check build (libfa_check.so) only: a device-side index or bounds
+                                  check failed; the access was skipped (fa_last_device_status) */
 } fa_status;
 
 /* Size of the built-in device scratch buffer of fa_bwd_noalloc (64 MiB per
@@ -246,10 +248,23 @@ size_t fa_bwd_workspace_size(int B, int H, int Sq, int D);
 size_t fa_bwd_workspace_size_ex(int B, int H, int Sq, int Sk, int D, int deterministic);
 
 /* Synchronises the current device, returns the status word recorded by
-   kernels since the last call (FA_OK or FA_ERR_TIMEOUT) and clears it.
-   FA_ERR_CUDA if the device cannot be queried. If `detail` is non-null it
-   receives 4 ints: code, linear block index, role (1 = loader, 2 = MMA
-   issuer, 3 = softmax/epilogue, 4 = self-test) and the block-loop iteration. */
+   kernels since the last call (FA_OK, FA_ERR_TIMEOUT or, in the check
+   build, FA_ERR_BOUNDS) and clears it. FA_ERR_CUDA if the device cannot be
+   queried. If `detail` is non-null it receives 4 ints: code, linear block
+   index, role (1 = loader, 2 = MMA issuer, 3 = softmax/epilogue, 4 =
+   self-test, 5 = bounds check) and the block-loop iteration (for a bounds
+   check: the number of the check site, see fa_common.cuh).
+   There is one status word per device, shared by every stream and thread
+   that uses the library on it: the first kernel to record a failure keeps
+   it until this call, which waits for all work on the device (not only one
+   stream) so that no kernel still running can record after the read.
+
+   The check build. libfa_check.so is the same library compiled with
+   FA_CHECK=1: the kernels test their own index arithmetic at the places
+   where it addresses memory (tile coordinates, TMEM columns, shared-memory
+   offsets, output and workspace indices against the sizes of the call). A
+   failed check records FA_ERR_BOUNDS and skips that access; nothing traps.
+   Results are the same as the normal build's; it runs slower. */
 int fa_last_device_status(int* detail);
 
 /* Self-test of failure detection (not a method step). Launches one block on

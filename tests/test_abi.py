@@ -26,6 +26,18 @@ def test_library_exports_every_declared_symbol(fa_lib):
         assert hasattr(fa_lib, name), name
 
 
+def test_check_build_exports_every_declared_symbol():
+    """libfa_check.so (FA_CHECK=1) is the same library: same entry points."""
+    from exact_io_aware_96_b200 import build
+    if not os.path.exists(fa.LIB_CHECK_PATH):
+        build.build(check=True)
+    L = ctypes.CDLL(fa.LIB_CHECK_PATH)
+    for name in declared_functions():
+        assert hasattr(L, name), name
+    L.fa_strerror.restype = ctypes.c_char_p
+    assert b"bounds check" in L.fa_strerror(-9)
+
+
 def test_version_and_strerror(fa_lib):
     assert fa.fa_version() >= 100
     for code in fa.STATUS:
@@ -251,3 +263,43 @@ def test_torch_helpers_marshal_well_formed_calls(monkeypatch):
     o8, _ = fa.forward_fp8(q8, k8, k8.clone(), 0.5, 0.25, 2.0, out_dtype=torch.float16)
     p = seen["fa_fwd_fp8_ex"]
     assert (p.Sq, p.Sk, p.o_dtype, p.v_descale) == (Sq, Sk, fa.FA_FP16, 2.0) and o8.dtype == torch.float16
+
+
+def test_backward_noalloc_helper_checks_and_marshals(monkeypatch):
+    """backward_noalloc (the torch helper over fa_bwd_noalloc) refuses CPU
+    tensors, buffers whose shape or dtype differ from what q and k imply, and
+    strided views (the entry point takes no strides); for well-formed buffers
+    it passes the sizes of q and k and the data pointers."""
+    import contextlib
+
+    import torch
+    f16 = torch.float16
+    B, Sq, Sk, H, D = 1, 8, 12, 2, 64
+    q = torch.zeros(B, Sq, H, D, dtype=f16)
+    k = torch.zeros(B, Sk, H, D, dtype=f16)
+    o = torch.zeros(B, Sq, H, D, dtype=f16)
+    lse = torch.zeros(B, H, Sq)
+    with pytest.raises(ValueError, match="CUDA device"):
+        fa.backward_noalloc(q, k, k, o, lse, o)
+    # pretend the tensors are on the GPU to reach the shape and layout checks
+    monkeypatch.setattr(torch.Tensor, "is_cuda", property(lambda self: True))
+    with pytest.raises(ValueError, match="v: expected shape"):
+        fa.backward_noalloc(q, k, torch.zeros(B, Sq, H, D, dtype=f16), o, lse, o)
+    with pytest.raises(TypeError, match="do: expected"):
+        fa.backward_noalloc(q, k, k, o, lse, o.bfloat16())
+    with pytest.raises(ValueError, match="lse: expected shape"):
+        fa.backward_noalloc(q, k, k, o, torch.zeros(B, H, Sk), o)
+    strided = torch.zeros(B, H, Sq, D, dtype=f16).transpose(1, 2)
+    with pytest.raises(ValueError, match="o must be a dense"):
+        fa.backward_noalloc(q, k, k, strided, lse, o)
+    with pytest.raises(ValueError, match="dk: expected shape"):
+        fa.backward_noalloc(q, k, k, o, lse, o, dk=torch.zeros(B, Sq, H, D, dtype=f16))
+    seen = {}
+    monkeypatch.setattr(fa, "_stream", lambda s: 0)
+    monkeypatch.setattr(torch.cuda, "device", lambda d: contextlib.nullcontext())
+    monkeypatch.setattr(fa, "fa_bwd_noalloc", lambda *a: seen.__setitem__("args", a) or 0)
+    dq, dk, dv = fa.backward_noalloc(q, k, k, o, lse, o, causal=True)
+    a = seen["args"]
+    assert a[0] == q.data_ptr() and a[6] == dq.data_ptr() and a[8] == dv.data_ptr()
+    assert a[9:17] == (B, H, Sq, Sk, D, D ** -0.5, 1, fa.FA_FP16)
+    assert dq.shape == q.shape and dk.shape == k.shape and dv.shape == k.shape
