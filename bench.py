@@ -78,7 +78,7 @@ def max_over_ranks(x: float, device=None) -> float:
 KERNEL_SOURCES = {
     "fa_bwd": ["fa_bwd.cuh", "fa_common.cuh", "sm100.cuh"],
     "fa_fwd_kernel": ["fa_fwd.cuh", "fa_common.cuh", "sm100.cuh"],
-    "fa_fwd_split_kernel": ["fa_fwd_split.cuh", "fa_fwd.cuh", "fa_common.cuh", "sm100.cuh"],
+    "fa_fwd_e4m3_kernel": ["fa_fwd_e4m3.cuh", "fa_fwd.cuh", "fa_common.cuh", "sm100.cuh"],
 }
 
 
@@ -350,7 +350,7 @@ def run_ours(args, w, causal):
     if t_bwd >= t_fwd:
         dom, dom_flops, dom_t = "fa_bwd (fa_bwd_pre + fa_bwd_main + fa_bwd_dq)", fb, t_bwd_max / args.steps
     else:
-        dom, dom_flops, dom_t = "fa_fwd_split_kernel", ff, t_fwd_max / args.steps
+        dom, dom_flops, dom_t = "fa_fwd_kernel", ff, t_fwd_max / args.steps
     achieved = dom_flops / dom_t / 1e12
     traffic = None
     tpath = os.path.join(ROOT, "profiles", "traffic.json")
@@ -508,7 +508,7 @@ def run_ours_fwd_e4m3(args, w, causal):
     if os.path.exists(tpath):
         with open(tpath) as f:
             ent = json.load(f).get("fa_fwd_kernel_e4m3")
-        if ent and ent.get("source_hash") == kernel_source_hash("fa_fwd_kernel"):
+        if ent and ent.get("source_hash") == kernel_source_hash("fa_fwd_e4m3_kernel"):
             traffic = ent.get("bytes_per_launch")
     result = {
         "metric": METRIC_E4M3, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -519,7 +519,7 @@ def run_ours_fwd_e4m3(args, w, causal):
                    "global_batch": w.B * world, "seq_len": w.S, "heads": w.H, "head_dim": w.D, "causal": causal,
                    "parallelism": f"dp{world} (independent heads, no collective)",
                    "l2": "flushed before every step (256 MiB write, outside the timed events)"},
-        "roofline": {"kernel": "fa_fwd_kernel<128, bf16 out, e4m3>", "bound": "tensor", "achieved": achieved,
+        "roofline": {"kernel": "fa_fwd_e4m3_kernel<128, bf16 out, e4m3>", "bound": "tensor", "achieved": achieved,
                      "peak": peak_tf, "unit": "TFLOP/s", "frac": achieved / peak_tf, "traffic": traffic,
                      "peak_source": f"{peaks_src} {key} x {E4M3_PER_BF16} (nominal fp8/bf16 ratio)"},
         "gpu_launches": args.steps,

@@ -12,7 +12,7 @@
 
 #include "fa.h"
 #include "fa_fwd.cuh"
-#include "fa_fwd_split.cuh"
+#include "fa_fwd_e4m3.cuh"
 #include "fa_bwd.cuh"
 
 namespace {
@@ -128,9 +128,9 @@ int prepare(F* fn, int smem_bytes, bool (&done)[kMaxDevices]) {
 
 template <int D, bool BF16>
 int launch_fwd(const fa_fwd_params* p, cudaStream_t stream) {
-  using L = fa::FwdSplitLayout<D>;
+  using L = fa::FwdLayout<D>;
   static bool done[kMaxDevices] = {};
-  auto* kern = &fa::fa_fwd_split_kernel<D, BF16>;
+  auto* kern = &fa::fa_fwd_kernel<D, BF16>;
   int st = prepare(kern, L::SMEM_ALLOC, done);
   if (st != FA_OK) return st;
   CUtensorMap mq, mk, mv;
@@ -160,9 +160,9 @@ int launch_fwd(const fa_fwd_params* p, cudaStream_t stream) {
 // e4m3 inputs: one kernel width (128 bytes = 128 columns) for every head_dim.
 template <bool OUT_BF16>
 int launch_fwd_fp8(const fa_fwd_fp8_params* p, cudaStream_t stream) {
-  using L = fa::FwdLayout<128, 1>;
+  using L = fa::FwdE4m3Layout<128, 1>;
   static bool done[kMaxDevices] = {};
-  auto* kern = &fa::fa_fwd_kernel<128, OUT_BF16, true>;
+  auto* kern = &fa::fa_fwd_e4m3_kernel<128, OUT_BF16>;
   int st = prepare(kern, L::SMEM_ALLOC, done);
   if (st != FA_OK) return st;
   CUtensorMap mq, mk, mv;
