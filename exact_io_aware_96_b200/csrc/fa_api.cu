@@ -89,14 +89,16 @@ int make_map(CUtensorMap* map, const fa_tensor& t, int B, int S, int H, int D, i
   return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
 
-// 2-D map over the fp32 dQ accumulator [rows][64], boxes of 32 rows x 32
-// floats (128 bytes) in the 128-byte swizzled shared-memory layout: the D = 64
-// backward stages dQ blocks that way and has the TMA add them.
-int make_dq_map(CUtensorMap* map, float* acc, int64_t rows) {
+// 2-D map over the fp32 dQ accumulator, [rows][cols] with cols innermost,
+// boxes of 32 rows x 32 floats (128 bytes) in the 128-byte swizzled
+// shared-memory layout: the backward stages dQ blocks that way and has the TMA
+// add them. D = 64: [B*H*Sq_pad][64]. D = 128: the accumulator is transposed,
+// [B*H*128][Sq_pad].
+int make_dq_map(CUtensorMap* map, float* acc, int64_t rows, int64_t cols) {
   auto fn = encode_fn();
   if (!fn) return FA_ERR_CUDA;
-  cuuint64_t dims[2] = {64, cuuint64_t(rows)};
-  cuuint64_t strides[1] = {64 * sizeof(float)};
+  cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
+  cuuint64_t strides[1] = {cuuint64_t(cols) * sizeof(float)};
   cuuint32_t box[2] = {32, 32};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, acc, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -248,18 +250,26 @@ int launch_bwd(const fa_bwd_params* p, cudaStream_t stream) {
     if ((st = prepare(&fa::fa_bwd_pre<D, BF16>, 0, done_pre)) != FA_OK) return st;
     if ((st = prepare(&fa::fa_bwd_dq<D, BF16>, 0, done_dq)) != FA_OK) return st;
     if ((st = prepare(&fa::fa_bwd_dq_sum<D, BF16>, 0, done_sum)) != FA_OK) return st;
+    static bool done_t[kMaxDevices] = {};
+    if ((st = prepare(&fa::fa_bwd_dq_t<BF16>, 0, done_t)) != FA_OK) return st;
   }
   const int64_t pre_threads = rows * G;
   fa::fa_bwd_pre<D, BF16><<<unsigned((pre_threads + 255) / 256), 256, 0, stream>>>(a);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   const unsigned grid = unsigned(int64_t((p->Sk + L::BN - 1) / L::BN) * p->B * p->H);
-  CUtensorMap mdq = mq;  // D = 128 does not read it
-  if (D == 64 && (st = make_dq_map(&mdq, a.dq_acc, rows)) != FA_OK) return st;
+  CUtensorMap mdq = mq;  // not read in deterministic mode
+  if (!p->deterministic) {
+    st = D == 64 ? make_dq_map(&mdq, a.dq_acc, rows, 64)
+                 : make_dq_map(&mdq, a.dq_acc, int64_t(p->B) * p->H * D, a.Sq_pad);
+    if (st != FA_OK) return st;
+  }
   kern<<<grid, L::kThreads, L::SMEM_ALLOC, stream>>>(mq, mk, mv, mdo, mdq, a);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   const int64_t dq_threads = int64_t(p->B) * p->H * p->Sq * G;
   if (a.dq_part != nullptr)
     fa::fa_bwd_dq_sum<D, BF16><<<unsigned((dq_threads + 255) / 256), 256, 0, stream>>>(a);
+  else if (D == 128)
+    fa::fa_bwd_dq_t<BF16><<<dim3(unsigned((p->Sq + 31) / 32), unsigned(p->B * p->H)), 256, 0, stream>>>(a);
   else
     fa::fa_bwd_dq<D, BF16><<<unsigned((dq_threads + 255) / 256), 256, 0, stream>>>(a);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;

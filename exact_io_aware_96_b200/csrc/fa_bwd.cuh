@@ -134,6 +134,50 @@ __global__ void __launch_bounds__(256) fa_bwd_dq(const BwdArgs a) {
 }
 
 // ------------------------------------------------ deterministic dq reduction
+// D = 128: the accumulator is [b][h][d][Sq_pad] (the main kernel adds dQ^T
+// blocks into it). One block of 256 threads per (b, h, 32 queries): the 128 x
+// 32 floats are read along the query axis into shared memory and written out
+// as dq rows of 128 head-dim values.
+template <bool BF16>
+__global__ void __launch_bounds__(256) fa_bwd_dq_t(const BwdArgs a) {
+  constexpr int D = 128;
+  __shared__ float tile[D][33];  // +1 column: the write-out reads hit different banks
+  const int bh = blockIdx.y;
+  const int h = bh % a.H;
+  const int b = bh / a.H;
+  const int i0 = blockIdx.x * 32;
+  if (!checked(b < a.B && i0 < a.Sq, 205)) return;
+  {
+    const int d = threadIdx.x >> 1, half = threadIdx.x & 1;
+    const float4* src = reinterpret_cast<const float4*>(a.dq_acc + (static_cast<int64_t>(bh) * D + d) * a.Sq_pad + i0 +
+                                                        16 * half);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float4 x = src[u];
+      tile[d][16 * half + 4 * u] = x.x;
+      tile[d][16 * half + 4 * u + 1] = x.y;
+      tile[d][16 * half + 4 * u + 2] = x.z;
+      tile[d][16 * half + 4 * u + 3] = x.w;
+    }
+  }
+  __syncthreads();
+  const float s = a.scale;
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    const int task = threadIdx.x + 256 * r;
+    const int ii = task >> 4, dc = task & 15;  // query row of the tile, 8-column group
+    const int i = i0 + ii;
+    if (i >= a.Sq || dc * 8 >= a.d) continue;
+    uint4 out;
+    out.x = sm100::pack2<BF16>(tile[8 * dc][ii] * s, tile[8 * dc + 1][ii] * s);
+    out.y = sm100::pack2<BF16>(tile[8 * dc + 2][ii] * s, tile[8 * dc + 3][ii] * s);
+    out.z = sm100::pack2<BF16>(tile[8 * dc + 4][ii] * s, tile[8 * dc + 5][ii] * s);
+    out.w = sm100::pack2<BF16>(tile[8 * dc + 6][ii] * s, tile[8 * dc + 7][ii] * s);
+    *reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(a.dq) + b * a.dq_sb + static_cast<int64_t>(i) * a.dq_ss +
+                              h * a.dq_sh + dc * 8) = out;
+  }
+}
+
 // dq = scale * sum over key blocks, in increasing key-block order, of the
 // dQ blocks the main kernel stored in their (query block, key block) slots.
 // A key block contributes to query block qb iff qb >= bwd_first_qblock(kvb),
@@ -655,14 +699,12 @@ __global__ void __launch_bounds__(448, 1)
           red_add_f32(p, x);
       };
       for (int i = 0; i < n; ++i) {
-        bool ok = __all_sync(0xffffffffu, wait_bar(dq_full, i & 1, abort_flag, kRoleSoftmax, i));
-        // The staged path synchronises the four drain warps on a named
-        // barrier, so they must all go on or all stop.
-        if constexpr (L::DQ_T && !DET) ok = named_bar_and(1, 128, ok);
+        const bool ok = __all_sync(0xffffffffu, wait_bar(dq_full, i & 1, abort_flag, kRoleSoftmax, i));
         if (!ok) break;
         tc_fence_after();
         const int qb = i_start + i;
         // block base: row0 of the accumulator, or the (qb, kvb) slot
+        // (D = 128 adds through the TMA and tmDQ and does not use `base`.)
         float* base = DET ? a.dq_part + ((static_cast<int64_t>(hb) * a.nqb + qb) * a.nkb + kvb) * (BM * D)
                           : a.dq_acc + (bh_row0 + static_cast<int64_t>(qb) * BM) * D;
         // Every write of this block lands in [base, base + BM * D); the check
@@ -697,28 +739,31 @@ __global__ void __launch_bounds__(448, 1)
               for (int c = 0; c < 32; ++c)
                 put(col + (32 * part + c) * D, __uint_as_float(v[part == 3 ? 0 : part][c]));
           } else {
-            // Quarter p (32 query rows) goes to staging buffer p & 1 as rows of
-            // 128 floats (each warp writes 128 contiguous bytes per row), then
-            // one thread has the TMA add the 16 KB into the accumulator, where
-            // the same 32 rows are contiguous. A buffer is rewritten only after
-            // the TMA has finished reading it.
-            const uint32_t stage0 = smem_u32(smem + L::OFF_DQS);
+            // The accumulator is kept transposed at D = 128, [b][h][d][Sq_pad]:
+            // this warp's 32 head-dim rows of quarter p (32 queries) are one
+            // 32 x 32-float box of it. The warp stages the box in the 128-byte
+            // swizzled layout (row d's 16-byte chunk c at d * 128 + ((c ^ (d %
+            // 8)) * 16): eight 16-byte stores per thread, no bank conflicts)
+            // and has the TMA add it through tmDQ. Each warp owns a quarter of
+            // each of the two staging buffers, so the four drain warps do not
+            // wait for one another. Y is released after the first quarter is
+            // staged and the last one read.
+            const int wq = warp & 3;
             auto store = [&](int part, const uint32_t (&x)[32]) {
-              const uint32_t buf = stage0 + (part & 1) * L::DQ_PART;
-              if (warp == 8 && lane == 0) bulk_wait_read1();  // the group that read this buffer last
+              uint8_t* buf = smem + L::OFF_DQS + (part & 1) * L::DQ_PART + wq * (32 * 128);
+              if (lane == 0) bulk_wait_read1();  // the reduction that read this buffer last
               __syncwarp();
-              named_bar_sync(1, 128);
+              const uint32_t rbase = smem_u32(buf) + lane * 128;
 #pragma unroll
-              for (int c = 0; c < 32; ++c) st_shared_f32(buf + (c * D + tr) * 4, __uint_as_float(x[c]));
+              for (int c = 0; c < 8; ++c)
+                st_shared_v4(rbase + ((c ^ (lane & 7)) << 4), x[4 * c], x[4 * c + 1], x[4 * c + 2], x[4 * c + 3]);
               fence_proxy_async_smem();
-            };
-            auto reduce = [&](int part) {
-              named_bar_sync(1, 128);
-              if (warp == 8 && lane == 0) {
-                if (checked(bh_row0 + static_cast<int64_t>(qb) * BM + 32 * part + 32 <=
-                                static_cast<int64_t>(a.B) * a.H * a.Sq_pad,
+              __syncwarp();
+              if (lane == 0) {
+                const int64_t drow = static_cast<int64_t>(hb) * D + 32 * wq;  // (b, h, d) row of the accumulator
+                if (checked(qb * BM + 32 * part + 32 <= a.Sq_pad && drow + 32 <= static_cast<int64_t>(a.B) * a.H * D,
                             214))
-                  bulk_reduce_add_f32(base + 32 * part * D, smem + L::OFF_DQS + (part & 1) * L::DQ_PART, L::DQ_PART);
+                  tma_reduce_add_2d(&tmDQ, buf, qb * BM + 32 * part, static_cast<int>(drow));
                 bulk_commit();
               }
             };
@@ -728,13 +773,9 @@ __global__ void __launch_bounds__(448, 1)
             reg_fence(v[0]);
             tc_fence_before();
             mbar_arrive(dq_free);  // Y may take dP^T(i+1) now
-            reduce(0);
             store(1, v[1]);
-            reduce(1);
             store(2, v[2]);
-            reduce(2);
             store(3, v[0]);
-            reduce(3);
           }
         } else {
           // lane = query row, columns = head_dim (64): the whole block fits in
@@ -796,8 +837,8 @@ __global__ void __launch_bounds__(448, 1)
     } else {
       drain(std::false_type{});
       // Let the TMA finish the last reductions before shared memory goes away
-      // (D = 128: warp 8 issued them; D = 64: lane 0 of each drain warp).
-      if (lane == 0 && (!L::DQ_T || warp == 8)) bulk_wait0();
+      // (lane 0 of each drain warp issued its own).
+      if (lane == 0) bulk_wait0();
     }
   }
 
