@@ -166,6 +166,11 @@ def clock_peak_pct(fwd_tf, bwd_tf, clk):
     return {"fwd": 100 * fwd_tf / peak, "bwd": 100 * bwd_tf / peak, "peak": peak, "sm_mhz": mhz}
 
 
+def dtype_name(dt) -> str:
+    import torch
+    return {torch.float16: "f16", torch.bfloat16: "bf16"}[dt]
+
+
 def flops(w, causal):
     return w.fwd_flops(causal), w.bwd_flops(causal)
 
@@ -230,11 +235,16 @@ def run_ours(args, w, causal):
     lse = torch.empty((B, H, S), dtype=torch.float32, device=dev)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     ws = fa.workspace_for(B, H, S, D, dev)
+    # The forward's key-range split, as the library chooses it for this shape.
+    fws = fa.fwd_workspace_for(B, H, S, S, D, causal, dev)
+    n_split = fa.fwd_workspace_size(B, H, S, S, D, causal, 0, dev)[1]
+    fsplit = 0 if fws is not None else -1
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
     def step():
-        fa.forward(q, k, v, causal=causal, scale=w.scale, out=o, lse=lse, stream=stream)
+        fa.forward(q, k, v, causal=causal, scale=w.scale, out=o, lse=lse, stream=stream, workspace=fws,
+                   split_ranks=fsplit)
         fa.backward(q, k, v, o, lse, do, causal=causal, scale=w.scale, dq=dq, dk=dk, dv=dv,
                     workspace=ws, stream=stream)
 
@@ -256,7 +266,8 @@ def run_ours(args, w, causal):
             flush.zero_()  # evict the inputs from L2 (outside the timed events)
             torch.cuda._sleep(PRE_STEP_SPIN_CYCLES)
             ev[i][0].record(stream)
-            fa.forward(q, k, v, causal=causal, scale=w.scale, out=o, lse=lse, stream=stream)
+            fa.forward(q, k, v, causal=causal, scale=w.scale, out=o, lse=lse, stream=stream, workspace=fws,
+                       split_ranks=fsplit)
             ev[i][1].record(stream)
             fa.backward(q, k, v, o, lse, do, causal=causal, scale=w.scale, dq=dq, dk=dk, dv=dv,
                         workspace=ws, stream=stream)
@@ -343,6 +354,19 @@ def run_ours(args, w, causal):
         del pipe
 
     peaks, peaks_src = load_peaks()
+    # Memory side of the same calls: the algorithmic bytes (every input read
+    # once, every output written once; the fp32 workspace is not counted)
+    # over the call's device time, against the measured copy bandwidth.
+    elt = q.element_size()
+    tens = B * S * H * D * elt
+    rows4 = B * H * S * 4
+    fwd_bytes = 4 * tens + rows4          # Q, K, V in; O, LSE out
+    bwd_bytes = 8 * tens + rows4          # Q, K, V, O, dO, LSE in; dQ, dK, dV out
+    fwd_gbs = fwd_bytes * args.steps / t_fwd_max / 1e9 * world
+    bwd_gbs = bwd_bytes * args.steps / t_bwd_max / 1e9 * world
+    hbm = {"fwd_bytes": fwd_bytes, "bwd_bytes": bwd_bytes, "fwd_gbs": fwd_gbs, "bwd_gbs": bwd_gbs,
+           "peak_gbs": peaks["hbm_gbs"], "fwd_frac": fwd_gbs / peaks["hbm_gbs"], "bwd_frac": bwd_gbs / peaks["hbm_gbs"],
+           "peak_source": f"{peaks_src} hbm_gbs"}
     timed_s = t_fwd + t_bwd
     sustained = timed_s > 1.0
     peak_tf = peaks.get("bf16_tflops_sustained" if sustained else "bf16_tflops")
@@ -365,11 +389,12 @@ def run_ours(args, w, causal):
     result = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": t_dev / args.steps * 1e3, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": f"{w.name}: B={w.B} H={w.H} S={w.S} D={w.D} bf16 causal={causal}, "
+        "scaling": "weak", "vs_baseline": None, "dtype": dtype_name(w.dtype), "data": "synthetic",
+        "config": {"workload": f"{w.name}: B={w.B} H={w.H} S={w.S} D={w.D} {dtype_name(w.dtype)} causal={causal}, "
                                "forward + backward per step",
                    "global_batch": w.B * world, "seq_len": w.S, "heads": w.H, "head_dim": w.D,
                    "causal": causal, "parallelism": f"dp{world} (independent heads, no collective)",
+                   "fwd_split_ranks": n_split,
                    "l2": "flushed before every step (256 MiB write, outside the timed events)"},
         "fwd_tflops": fwd_tf, "bwd_tflops": bwd_tf,
         "fwd_us": t_fwd_max / args.steps * 1e6, "bwd_us": t_bwd_max / args.steps * 1e6,
@@ -385,6 +410,7 @@ def run_ours(args, w, causal):
         "roofline": {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
                      "frac": achieved / peak_tf, "traffic": traffic,
                      "peak_source": f"{peaks_src} {'bf16_tflops_sustained' if sustained else 'bf16_tflops'}"},
+        "hbm": hbm,
         "gpu_launches": 4 * args.steps,
         "clocks": clocks.summary(),
         "wall_s_timed_region": wall,

@@ -5,10 +5,15 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
+#include <atomic>
+#include <chrono>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <functional>
 #include <mutex>
+#include <vector>
 
 #include "fa.h"
 #include "fa_fwd.cuh"
@@ -128,6 +133,162 @@ int prepare(F* fn, int smem_bytes, bool (&done)[kMaxDevices]) {
   return FA_OK;
 }
 
+// ------------------------------------------------------- key-range split plan
+// Workspace of a split over the first n_split ranks: tickets (one u64 per
+// split (b, h, rank)), then (m, l) per row and the fp32 O partial per row of
+// every split CTA; sections 256-byte aligned.
+struct SplitLayout {
+  uint64_t off_ml, off_o, bytes;
+};
+uint64_t round256(uint64_t x) { return (x + 255) / 256 * 256; }
+SplitLayout split_layout(int B, int H, int n_split, int Dk) {
+  const uint64_t pairs = uint64_t(B) * H * n_split;
+  const uint64_t ctas = 2 * pairs;
+  SplitLayout l;
+  l.off_ml = round256(pairs * 8);
+  l.off_o = l.off_ml + round256(ctas * 256 * 8);
+  l.bytes = n_split > 0 ? l.off_o + ctas * 256 * uint64_t(Dk) * 4 : 0;
+  return l;
+}
+
+int sm_count() {
+  static int count[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+  if (count[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    count[dev] = n;
+  }
+  return count[dev];
+}
+
+// A split plan: n_split ranks split, and the grid's unit order (see
+// FwdArgs::order), longest unit first.
+struct SplitPlan {
+  int ns = 0;
+  int units = 0;
+  uint8_t order[2 * fa::FwdArgs::kMaxSplitRanks] = {};
+};
+
+// Unit costs in 128 x 128 tile-blocks: a CTA's key blocks over both tiles,
+// plus a start-up cost (loading Q, filling the pipeline, the epilogue), plus
+// for a split half the exchange through the workspace and the merge. The
+// constants are fitted to per-CTA timings of the kernel on B200.
+constexpr double kSplitStart = 3.0;
+double split_merge_cost(int Dk) { return Dk <= 64 ? 4.0 : 5.0; }
+
+void split_costs(const int* c0, const int* c1, int r, double merge, double* whole, double* h0, double* h1) {
+  const int hs = (std::max(c0[r], c1[r]) + 1) / 2;
+  *whole = kSplitStart + c0[r] + c1[r];
+  *h0 = kSplitStart + merge + std::min(c0[r], hs) + std::min(c1[r], hs);
+  *h1 = kSplitStart + merge + std::max(0, c0[r] - hs) + std::max(0, c1[r] - hs);
+}
+
+// The order for `ns` split ranks: units sorted by cost, longest first (ties
+// in rank, then half order), so that CTAs starting in grid order on
+// whichever SM frees first is longest-processing-time-first list scheduling.
+SplitPlan split_order(const int* c0, const int* c1, int nq, int ns, double merge) {
+  SplitPlan p;
+  p.ns = ns;
+  std::vector<std::pair<double, int>> u;
+  for (int r = 0; r < nq; ++r) {
+    double w, a, b;
+    split_costs(c0, c1, r, merge, &w, &a, &b);
+    if (r < ns) {
+      u.push_back({a, r * 3 + 1});
+      u.push_back({b, r * 3 + 2});
+    } else {
+      u.push_back({w, r * 3});
+    }
+  }
+  std::stable_sort(u.begin(), u.end(), [](const std::pair<double, int>& x, const std::pair<double, int>& y) {
+    return x.first > y.first;
+  });
+  p.units = int(u.size());
+  for (size_t i = 0; i < u.size(); ++i) p.order[i] = uint8_t(u[i].second);
+  return p;
+}
+
+// Finish time of the plan's grid: CTAs start in grid order on whichever SM
+// frees first, one CTA per SM.
+double split_makespan(const int* c0, const int* c1, const SplitPlan& p, int HB, int sms, double merge) {
+  std::vector<double> heap(size_t(sms), 0.0);  // min-heap of SM free times
+  std::make_heap(heap.begin(), heap.end(), std::greater<double>());
+  for (int i = 0; i < p.units; ++i) {
+    const int r = p.order[i] / 3, kind = p.order[i] % 3;
+    double w, a, b;
+    split_costs(c0, c1, r, merge, &w, &a, &b);
+    const double cost = kind == 0 ? w : (kind == 1 ? a : b);
+    for (int j = 0; j < HB; ++j) {
+      std::pop_heap(heap.begin(), heap.end(), std::greater<double>());
+      heap.back() += cost;
+      std::push_heap(heap.begin(), heap.end(), std::greater<double>());
+    }
+  }
+  return *std::max_element(heap.begin(), heap.end());
+}
+
+// The plan for split_ranks (see fa_fwd_params): -1 none, k > 0 min(k, ranks),
+// 0 the estimate's best (kept only if it beats the unsplit grid by more than
+// 5%). No split past kMaxSplitRanks ranks. Automatic plans are cached per
+// shape.
+SplitPlan plan_split(int B, int H, int Sq, int Sk, int Dk, int causal, int split_ranks) {
+  const int nq = (Sq + 255) / 256;
+  SplitPlan none;
+  if (split_ranks < 0 || nq > fa::FwdArgs::kMaxSplitRanks) return none;
+  std::vector<int> c0(static_cast<size_t>(nq)), c1(static_cast<size_t>(nq));
+  for (int r = 0; r < nq; ++r) {
+    const int qb = causal ? nq - 1 - r : r;
+    c0[size_t(r)] = fa::fwd_kv_blocks(qb * 256, Sq, Sk, causal);
+    c1[size_t(r)] = fa::fwd_kv_blocks(qb * 256 + 128, Sq, Sk, causal);
+  }
+  const double merge = split_merge_cost(Dk);
+  if (split_ranks > 0) return split_order(c0.data(), c1.data(), nq, std::min(split_ranks, nq), merge);
+  const int sms = sm_count();
+  const int64_t HB = int64_t(B) * H;
+  if (sms <= 0 || HB * nq >= 4 * int64_t(sms)) return none;
+  struct Entry {
+    int B, H, Sq, Sk, Dk, causal, sms;
+    SplitPlan plan;
+  };
+  static Entry cache[32];
+  static int cache_n = 0, cache_next = 0;
+  static std::mutex mu;
+  {
+    std::lock_guard<std::mutex> g(mu);
+    for (int i = 0; i < cache_n; ++i) {
+      const Entry& e = cache[i];
+      if (e.B == B && e.H == H && e.Sq == Sq && e.Sk == Sk && e.Dk == Dk && e.causal == causal && e.sms == sms)
+        return e.plan;
+    }
+  }
+  SplitPlan best = split_order(c0.data(), c1.data(), nq, 0, merge);
+  const double base = split_makespan(c0.data(), c1.data(), best, int(HB), sms, merge);
+  double best_t = base;
+  for (int ns = 1; ns <= nq; ++ns) {
+    const SplitPlan p = split_order(c0.data(), c1.data(), nq, ns, merge);
+    const double t = split_makespan(c0.data(), c1.data(), p, int(HB), sms, merge);
+    if (t < best_t) {
+      best_t = t;
+      best = p;
+    }
+  }
+  if (best_t > 0.95 * base) best = none;
+  std::lock_guard<std::mutex> g(mu);
+  cache[cache_next] = Entry{B, H, Sq, Sk, Dk, causal, sms, best};
+  cache_next = (cache_next + 1) % 32;
+  cache_n = std::min(cache_n + 1, 32);
+  return best;
+}
+
+// Distinct for every launch of the split forward (the tickets compare it).
+unsigned long long next_epoch() {
+  static std::atomic<unsigned long long> epoch{
+      (uint64_t(std::chrono::steady_clock::now().time_since_epoch().count()) * 0x9E3779B97F4A7C15ull) | 1ull};
+  return epoch.fetch_add(2);
+}
+
 template <int D, bool BF16>
 int launch_fwd(const fa_fwd_params* p, cudaStream_t stream) {
   using L = fa::FwdLayout<D>;
@@ -139,7 +300,7 @@ int launch_fwd(const fa_fwd_params* p, cudaStream_t stream) {
   if ((st = make_map(&mq, p->q, p->B, p->Sq, p->H, p->D, p->dtype, 128)) != FA_OK) return st;
   if ((st = make_map(&mk, p->k, p->B, p->Sk, p->H, p->D, p->dtype, 128)) != FA_OK) return st;
   if ((st = make_map(&mv, p->v, p->B, p->Sk, p->H, p->D, p->dtype, 128)) != FA_OK) return st;
-  fa::FwdArgs a;
+  fa::FwdArgs a{};
   a.o = p->o.ptr;
   a.lse = p->lse;
   a.o_sb = p->o.stride_b;
@@ -154,7 +315,22 @@ int launch_fwd(const fa_fwd_params* p, cudaStream_t stream) {
   a.causal = p->causal;
   a.n_qblocks = (p->Sq + 255) / 256;
   a.d = p->D;
-  const unsigned grid = unsigned(int64_t(a.n_qblocks) * p->B * p->H);
+  if (p->workspace != nullptr) {
+    const SplitPlan plan = plan_split(p->B, p->H, p->Sq, p->Sk, D, p->causal, p->split_ranks);
+    const int ns = plan.ns;
+    const SplitLayout sl = split_layout(p->B, p->H, ns, D);
+    if (ns > 0) {
+      if (p->workspace_bytes < sl.bytes) return FA_ERR_WORKSPACE;
+      uint8_t* ws = static_cast<uint8_t*>(p->workspace);
+      a.n_split = ns;
+      std::memcpy(a.order, plan.order, sizeof(a.order));
+      a.tickets = reinterpret_cast<unsigned long long*>(ws);
+      a.part_ml = reinterpret_cast<float2*>(ws + sl.off_ml);
+      a.part_o = reinterpret_cast<float*>(ws + sl.off_o);
+      a.epoch = next_epoch();
+    }
+  }
+  const unsigned grid = unsigned(int64_t(a.n_qblocks + a.n_split) * p->B * p->H);
   kern<<<grid, L::kThreads, L::SMEM_ALLOC, stream>>>(mq, mk, mv, a);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
@@ -171,7 +347,7 @@ int launch_fwd_fp8(const fa_fwd_fp8_params* p, cudaStream_t stream) {
   if ((st = make_map(&mq, p->q, p->B, p->Sq, p->H, p->D, kE4M3, 128)) != FA_OK) return st;
   if ((st = make_map(&mk, p->k, p->B, p->Sk, p->H, p->D, kE4M3, 128)) != FA_OK) return st;
   if ((st = make_map(&mv, p->v, p->B, p->Sk, p->H, p->D, kE4M3, 128)) != FA_OK) return st;
-  fa::FwdArgs a;
+  fa::FwdArgs a{};
   a.o = p->o.ptr;
   a.lse = p->lse;
   a.o_sb = p->o.stride_b;
@@ -335,6 +511,7 @@ int fa_fwd_ex(const fa_fwd_params* p, fa_stream_t stream) {
     if ((st = check_view(*v)) != FA_OK) return st;
   if (p->lse == nullptr) return FA_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(p->lse) & 3u) return FA_ERR_MISALIGNED;
+  if (p->workspace != nullptr && (reinterpret_cast<uintptr_t>(p->workspace) & 255u)) return FA_ERR_MISALIGNED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   // head_dim <= 64 runs the 64-column kernels, <= 128 the 128-column ones;
   // the tensor maps read the columns past head_dim as zeros.
@@ -406,6 +583,19 @@ int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
   p.causal = causal;
   p.o_dtype = o_dtype;
   return fa_fwd_fp8_ex(&p, stream);
+}
+
+size_t fa_fwd_workspace_size_ex(int B, int H, int Sq, int Sk, int D, int causal, int split_ranks, int* n_split) {
+  if (n_split != nullptr) *n_split = 0;
+  if (check_common(B, H, Sq, Sk, D, 1.f, causal, FA_BF16) != FA_OK) return 0;
+  const int Dk = D <= 64 ? 64 : 128;
+  const int ns = plan_split(B, H, Sq, Sk, Dk, causal, split_ranks).ns;
+  if (n_split != nullptr) *n_split = ns;
+  return size_t(split_layout(B, H, ns, Dk).bytes);
+}
+
+size_t fa_fwd_workspace_size(int B, int H, int Sq, int Sk, int D, int causal) {
+  return fa_fwd_workspace_size_ex(B, H, Sq, Sk, D, causal, 0, nullptr);
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int Sq, int D) {

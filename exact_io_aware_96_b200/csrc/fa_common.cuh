@@ -112,6 +112,21 @@ struct FwdArgs {
   float o_scale;     // factor applied to O with 1/l: 1, or V's descale factor for e4m3 inputs
   int causal;
   int n_qblocks;     // ceil(Sq / 256)
+  // Key-range split (fa_fwd_kernel only; 0 elsewhere). The first n_split
+  // ranks (the heaviest query blocks when causal) each run as two CTAs, one
+  // per half of the key blocks; the two leave unnormalised partial results in
+  // the workspace and the second to finish merges them. 0: every CTA covers
+  // its whole key range and the grid is rank-major. Otherwise the grid runs
+  // the units order[0 .. n_qblocks + n_split) (B * H CTAs each), every entry
+  // rank * 3 + kind (kind 0: the whole rank, 1 and 2: its first and second
+  // half), longest first.
+  static constexpr int kMaxSplitRanks = 64;
+  int n_split;
+  uint8_t order[2 * kMaxSplitRanks];
+  float* part_o;                // fp32 [split CTA][256 rows][D]: unnormalised O
+  float2* part_ml;              // [split CTA][256 rows]: (running max m, row sum l), base 2
+  unsigned long long* tickets;  // [split pair]: the epoch of the first of its two CTAs to finish
+  unsigned long long epoch;     // distinct for every launch
 };
 
 // First query block that key block kvb contributes to: with a causal mask,

@@ -66,13 +66,13 @@
 namespace fa {
 
 // Number of 128-key blocks that rows [r0, r0 + 128) of the query range need.
-__device__ __forceinline__ int fwd_kv_blocks(int r0, int Sq, int Sk, int causal) {
+__host__ __device__ inline int fwd_kv_blocks(int r0, int Sq, int Sk, int causal) {
   if (r0 >= Sq) return 0;
   const int nk = (Sk + 127) / 128;
   if (!causal) return nk;
-  const int last = min(r0 + 127, Sq - 1) + (Sk - Sq);
+  const int last = (r0 + 127 < Sq - 1 ? r0 + 127 : Sq - 1) + (Sk - Sq);
   if (last < 0) return 0;
-  return min(nk, last / 128 + 1);
+  return nk < last / 128 + 1 ? nk : last / 128 + 1;
 }
 
 // ESZ: bytes per Q/K/V element (2 for fp16/bf16, 1 for e4m3).
@@ -138,6 +138,134 @@ __device__ __forceinline__ void fwd_exp32(const uint32_t (&sv)[32], int col0, in
   }
 }
 
+// Epilogue of a CTA that covers one half of its rows' key blocks (FwdArgs::
+// n_split). Every softmax warp of the CTA calls it. The CTA's partial result
+// for a row, (m, l = l_0 + l_1, unnormalised O), is exact for that half of the
+// keys; two halves merge exactly:
+//   m = max(m_a, m_b),  l = l_a 2^(m_a - m) + l_b 2^(m_b - m),
+//   O = (O_a 2^(m_a - m) + O_b 2^(m_b - m)) / l,
+// the same rescaling the online softmax applies from one key block to the
+// next ([P4] §3.1), here between the two halves. Each CTA writes its partial
+// into its workspace slot; the 16 softmax warps meet; one thread fences and
+// swaps the pair's ticket to this launch's epoch; the CTA that finds the
+// epoch already there (the second to finish) fences again and reads its
+// partner's partial through L2, then writes O and LSE. The barrier orders the
+// other threads' partial stores before that thread's fence (fences are
+// cumulative), so one fence per CTA suffices.
+// Partial O layout: float4 units [CTA][tile][D / 4][128 rows], so a warp's
+// stores and loads of one 4-column group cover 512 contiguous bytes.
+template <int D, bool BF16>
+__device__ __forceinline__ void fwd_split_epilogue(const FwdArgs& a, uint8_t* flag_smem, float* lsum, uint64_t* o_final,
+                                                   volatile int* abort_flag, uint32_t tO, bool ok, int t, int c, int r,
+                                                   int pair_bar, int n, float m, float l, int pair, int cta, int pcta,
+                                                   int b, int h, int row, int r0) {
+  using namespace sm100;
+  constexpr int kSplitBar = 9;  // named barrier of the 16 softmax warps
+  const bool rows = r0 < a.Sq;  // the same for both warps of a pair
+  bool go = ok && !*abort_flag;
+  float lt = 0.f;
+  if (rows) {
+    lsum[(t * 2 + c) * 128 + r] = l;
+    go = named_bar_and(pair_bar, 64, go);
+    lt = l + lsum[(t * 2 + (c ^ 1)) * 128 + r];
+  }
+  const int n_ctas = 2 * a.n_split * a.H * a.B;
+  // first float4 of this thread's columns in a CTA's partial O; step 128 per 4 columns
+  auto o_base = [&](int k) {
+    return reinterpret_cast<float4*>(a.part_o) + (static_cast<int64_t>(k) * 2 + t) * (D / 4) * 128 +
+           static_cast<int64_t>(c * (D / 8)) * 128 + r;
+  };
+  bool have_o = false;  // O_t holds this CTA's sums (n > 0 and its MMAs are done)
+  if (go && rows && n > 0) {
+    have_o = __all_sync(0xffffffffu, wait_bar(o_final, 0, abort_flag, kRoleSoftmax, n));
+    go = have_o;
+    if (have_o) tc_fence_after();
+  }
+  // (Conditions around tcgen05.ld are warp-uniform: the load is collective.)
+  if (__all_sync(0xffffffffu, go && rows && checked(cta < n_ctas, 110))) {
+    float4* po = o_base(cta);
+#pragma unroll 1
+    for (int q = 0; q < D / 64; ++q) {
+      uint32_t ov[32];
+      if (have_o) {
+        tmem_ld32(tO + 32 * q, ov);
+        tmem_ld_wait();
+        reg_fence(ov);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) ov[i] = 0u;
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        po[(8 * q + i) * 128] = make_float4(__uint_as_float(ov[4 * i]), __uint_as_float(ov[4 * i + 1]),
+                                            __uint_as_float(ov[4 * i + 2]), __uint_as_float(ov[4 * i + 3]));
+    }
+    if (c == 0) a.part_ml[static_cast<int64_t>(cta) * 256 + t * 128 + r] = make_float2(m, lt);
+  }
+  go = named_bar_and(kSplitBar, 512, go);
+  volatile uint32_t* second_flag = reinterpret_cast<volatile uint32_t*>(flag_smem);
+  if (threadIdx.x == 0) {
+    uint32_t second = 0;
+    if (go && checked(pair < a.n_split * a.H * a.B, 112)) {
+      __threadfence();
+      second = atomicExch(&a.tickets[pair], a.epoch) == a.epoch;
+      if (second) __threadfence();
+    }
+    *second_flag = second;
+  }
+  named_bar_sync(kSplitBar, 512);
+  if (!__all_sync(0xffffffffu, go && rows && *second_flag && checked(pcta >= 0 && pcta < n_ctas, 111))) return;
+  const float2 mo = __ldcg(a.part_ml + static_cast<int64_t>(pcta) * 256 + t * 128 + r);  // the partner's (m, l)
+  const float mn = fmaxf(m, mo.x);
+  const float as = (m == -INFINITY) ? 0.f : ex2(m - mn);
+  const float ao = (mo.x == -INFINITY) ? 0.f : ex2(mo.x - mn);
+  // Products rounded separately and then added (no fused multiply-add), so
+  // the result is the same whichever of the two CTAs merges.
+  const float lsum_all = __fadd_rn(__fmul_rn(lt, as), __fmul_rn(mo.y, ao));
+  const bool has = (mn != -INFINITY) && lsum_all > 0.f;  // false only for rows with no allowed key
+  const float inv = has ? a.o_scale / lsum_all : 0.f;
+  const float ws = as * inv, wo = ao * inv;
+  const bool valid = row < a.Sq;
+  const int cb = c * (D / 2);  // first O column of this half
+  const float4* ppo = o_base(pcta);
+  uint16_t* orow = reinterpret_cast<uint16_t*>(a.o) + static_cast<int64_t>(b) * a.o_sb +
+                   static_cast<int64_t>(row) * a.o_ss + static_cast<int64_t>(h) * a.o_sh;
+#pragma unroll 1
+  for (int q = 0; q < D / 64; ++q) {
+    float4 pv[8];  // the partner's 32 columns, loaded while this CTA's come out of TMEM
+#pragma unroll
+    for (int i = 0; i < 8; ++i) pv[i] = __ldcg(ppo + (8 * q + i) * 128);
+    uint32_t ov[32];
+    if (have_o) {
+      tmem_ld32(tO + 32 * q, ov);
+      tmem_ld_wait();
+      reg_fence(ov);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) ov[i] = 0u;
+    }
+    auto mix = [&](uint32_t own, float other) {
+      return __fadd_rn(__fmul_rn(__uint_as_float(own), ws), __fmul_rn(other, wo));
+    };
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      pk[2 * i] = pack2<BF16>(mix(ov[4 * i], pv[i].x), mix(ov[4 * i + 1], pv[i].y));
+      pk[2 * i + 1] = pack2<BF16>(mix(ov[4 * i + 2], pv[i].z), mix(ov[4 * i + 3], pv[i].w));
+    }
+    if (valid) {
+      uint4* dst = reinterpret_cast<uint4*>(orow + cb + 32 * q);
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (cb + 32 * q + 8 * i < a.d && checked(row < a.Sq && b < a.B && h < a.H, 107))
+          dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+    }
+  }
+  if (valid && c == 0 && checked(b < a.B && h < a.H && row < a.Sq, 108))
+    a.lse[(static_cast<int64_t>(b) * a.H + h) * a.Sq + row] =
+        has ? (mn + __log2f(lsum_all)) * 0.69314718055994531f : -INFINITY;
+}
+
 // Q, K, V and O are fp16 (BF16 = false) or bf16 (BF16 = true).
 template <int D, bool BF16>
 __global__ void __launch_bounds__(576, 1)
@@ -174,17 +302,44 @@ __global__ void __launch_bounds__(576, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // Linear block order: all heads' heaviest query blocks first (causal).
+  // Grid order: unit-major over (b, h). Ranks count query blocks from the
+  // last one (the most key blocks) down with a causal mask, from the first
+  // without. Unsplit, unit = rank. With a split the units come from
+  // FwdArgs::order, longest first: a whole rank, or one half of a split rank
+  // (half 0: key blocks [0, hs), half 1: [hs, n), hs = ceil(n / 2) of the
+  // block's longer tile).
   const int hb_count = a.H * a.B;
-  const int rank = blockIdx.x / hb_count;
+  const int unit = blockIdx.x / hb_count;
   const int hb = blockIdx.x % hb_count;
+  int rank = unit, half = 0;
+  bool split = false;
+  if (a.n_split > 0) {
+    const int e = a.order[unit < 2 * FwdArgs::kMaxSplitRanks ? unit : 0];
+    checked(unit < a.n_qblocks + a.n_split && unit < 2 * FwdArgs::kMaxSplitRanks, 113);
+    rank = e / 3;
+    split = (e % 3) != 0;
+    half = split ? (e % 3) - 1 : 0;
+  }
   const int h = hb % a.H;
   const int b = hb / a.H;
   const int qb = a.causal ? (a.n_qblocks - 1 - rank) : rank;
   const int q0 = qb * 256;
+  // This CTA's key blocks of tile t: [jlo, jlo + nkv[t]).
   int nkv[2];
   nkv[0] = fwd_kv_blocks(q0, a.Sq, a.Sk, a.causal);
   nkv[1] = fwd_kv_blocks(q0 + 128, a.Sq, a.Sk, a.causal);
+  int jlo = 0;
+  if (split) {
+    const int hs = (max(nkv[0], nkv[1]) + 1) / 2;
+    if (half == 0) {
+      nkv[0] = min(nkv[0], hs);
+      nkv[1] = min(nkv[1], hs);
+    } else {
+      jlo = hs;
+      nkv[0] = max(0, nkv[0] - hs);
+      nkv[1] = max(0, nkv[1] - hs);
+    }
+  }
   const int nmax = max(nkv[0], nkv[1]);
 
   if (threadIdx.x == 0) {
@@ -239,17 +394,19 @@ __global__ void __launch_bounds__(576, 1)
         const uint32_t ph = (j / S) & 1;
         if (!wait_bar(&k_empty[st], ph ^ 1, abort_flag, kRoleLoader, j)) break;
         mbar_arrive_expect_tx(&k_full[st], L::TILE);
-        checked(j * 128 < a.Sk && st < S, 102);
+        checked((jlo + j) * 128 < a.Sk && st < S, 102);
         for (int kb = 0; kb < L::KB; ++kb)
-          tma_load_4d(smem + L::OFF_K + st * L::TILE + kb * L::BLK, &tmK, &k_full[st], kb * KCOL, j * 128, h, b);
+          tma_load_4d(smem + L::OFF_K + st * L::TILE + kb * L::BLK, &tmK, &k_full[st], kb * KCOL, (jlo + j) * 128, h,
+                      b);
         if (!wait_bar(&v_empty[st], ph ^ 1, abort_flag, kRoleLoader, j)) {
           ++j;  // K_j was issued
           break;
         }
         mbar_arrive_expect_tx(&v_full[st], L::TILE);
-        checked(j * 128 < a.Sk && st < S, 102);
+        checked((jlo + j) * 128 < a.Sk && st < S, 102);
         for (int kb = 0; kb < L::KB; ++kb)
-          tma_load_4d(smem + L::OFF_V + st * L::TILE + kb * L::BLK, &tmV, &v_full[st], kb * KCOL, j * 128, h, b);
+          tma_load_4d(smem + L::OFF_V + st * L::TILE + kb * L::BLK, &tmV, &v_full[st], kb * KCOL, (jlo + j) * 128, h,
+                      b);
       }
       if (*abort_flag) {
         // Let the copies already issued land before the CTA exits. A V copy
@@ -407,7 +564,7 @@ __global__ void __launch_bounds__(576, 1)
       // `ok` false here: a wait of the previous block ran out; this warp goes
       // straight to the pair barrier, which then ends both warps.
       const bool ready = ok && __all_sync(0xffffffffu, wait_bar(&s_full[t], j & 1, abort_flag, kRoleSoftmax, j));
-      const int k0 = j * 128 + 64 * c;  // first key of this half
+      const int k0 = (jlo + j) * 128 + 64 * c;  // first key of this half
       const bool masked = k0 + 64 > a.Sk || (a.causal && k0 + 63 > r0 + off);
       int lim = a.Sk - 1 - k0;  // last allowed column of this half
       if (a.causal) lim = min(lim, row + off - k0);
@@ -522,7 +679,12 @@ __global__ void __launch_bounds__(576, 1)
     // Epilogue: O = O_t / (l_0 + l_1), LSE = ln2 * (m + log2(l_0 + l_1)).
     // Both warps of the pair arrive here with the same `ok` (the loop's
     // barrier ANDs it), so both take the barrier below or neither does.
-    if (r0 < a.Sq) {
+    if (split) {
+      // Workspace slots: split rank `rank`, half `half`, (b, h) `hb`.
+      fwd_split_epilogue<D, BF16>(a, smem + L::OFF_MISC + 8, lsum, &o_final[t], abort_flag, tO, ok, t, c, r, pair_bar,
+                                  n, m, l, rank * hb_count + hb, (2 * rank + half) * hb_count + hb,
+                                  (2 * rank + 1 - half) * hb_count + hb, b, h, row, r0);
+    } else if (r0 < a.Sq) {
       lsum[(t * 2 + c) * 128 + r] = l;
       const bool go = named_bar_and(pair_bar, 64, ok && !*abort_flag);
       const bool valid = row < a.Sq;

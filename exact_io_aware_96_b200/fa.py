@@ -22,6 +22,8 @@ LIB_CHECK_PATH = os.path.join(_HERE, "libfa_check.so")
 
 FA_FP16, FA_BF16 = 0, 1
 FA_OK = 0
+FA_ERR_MISALIGNED = -3
+FA_ERR_WORKSPACE = -7
 STATUS = {
     0: "FA_OK", -1: "FA_ERR_INVALID_ARG", -2: "FA_ERR_UNSUPPORTED", -3: "FA_ERR_MISALIGNED",
     -4: "FA_ERR_CUDA", -5: "FA_ERR_TIMEOUT", -6: "FA_ERR_NOT_IMPLEMENTED", -7: "FA_ERR_WORKSPACE",
@@ -29,6 +31,7 @@ STATUS = {
 }
 FA_NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 EXPORTED = ("fa_fwd", "fa_fwd_ex", "fa_fwd_fp8", "fa_fwd_fp8_ex", "fa_bwd", "fa_bwd_ex", "fa_bwd_noalloc",
+            "fa_fwd_workspace_size", "fa_fwd_workspace_size_ex",
             "fa_bwd_workspace_size", "fa_bwd_workspace_size_ex", "fa_selftest_wait_timeout",
             "fa_last_device_status", "fa_strerror", "fa_version")
 
@@ -43,7 +46,9 @@ class FwdParams(ctypes.Structure):
                 ("lse", ctypes.c_void_p),
                 ("B", ctypes.c_int), ("H", ctypes.c_int), ("Sq", ctypes.c_int), ("Sk", ctypes.c_int),
                 ("D", ctypes.c_int), ("scale", ctypes.c_float), ("causal", ctypes.c_int),
-                ("dtype", ctypes.c_int)]
+                ("dtype", ctypes.c_int),
+                ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+                ("split_ranks", ctypes.c_int)]
 
 
 class FwdFp8Params(ctypes.Structure):
@@ -105,6 +110,10 @@ def lib():
         L.fa_bwd_ex.restype = i
         L.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp]
         L.fa_bwd_noalloc.restype = i
+        L.fa_fwd_workspace_size.argtypes = [i, i, i, i, i, i]
+        L.fa_fwd_workspace_size.restype = sz
+        L.fa_fwd_workspace_size_ex.argtypes = [i, i, i, i, i, i, i, ctypes.POINTER(ctypes.c_int)]
+        L.fa_fwd_workspace_size_ex.restype = sz
         L.fa_bwd_workspace_size.argtypes = [i, i, i, i]
         L.fa_bwd_workspace_size.restype = sz
         L.fa_bwd_workspace_size_ex.argtypes = [i, i, i, i, i, i]
@@ -235,8 +244,28 @@ def _stream(stream) -> int:
     return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
 
 
-def forward(q, k, v, causal=False, scale=None, out=None, lse=None, stream=None):
-    """O, LSE = attention(q, k, v) on [B, S, H, D] CUDA tensors (strided views allowed)."""
+def fwd_workspace_size(B, H, Sq, Sk, D, causal, split_ranks=0, device=None):
+    """(bytes, split ranks) of the forward's key-range split on `device`
+    (default: the current one); (0, 0) when no split is chosen."""
+    ns = ctypes.c_int(0)
+    with torch.cuda.device(device if device is not None else torch.cuda.current_device()):
+        n = lib().fa_fwd_workspace_size_ex(B, H, Sq, Sk, D, int(bool(causal)), int(split_ranks), ctypes.byref(ns))
+    return int(n), ns.value
+
+
+def fwd_workspace_for(B, H, Sq, Sk, D, causal, device, split_ranks=0):
+    """A workspace for forward(..., workspace=...), or None when no split is chosen."""
+    n, _ = fwd_workspace_size(B, H, Sq, Sk, D, causal, split_ranks, device)
+    return torch.empty(n, dtype=torch.uint8, device=device) if n else None
+
+
+def forward(q, k, v, causal=False, scale=None, out=None, lse=None, stream=None, workspace=None, split_ranks=0):
+    """O, LSE = attention(q, k, v) on [B, S, H, D] CUDA tensors (strided views allowed).
+
+    split_ranks: 0 lets the library choose a key-range split of the heaviest
+    query blocks (it then needs a workspace, taken from torch's allocator
+    unless one is given), k > 0 splits the first k query-block ranks, -1
+    never splits."""
     B, Sq, H, D, Sk = _dims(q, k)
     dt = _dtype_code(q)
     dev = q.device
@@ -250,8 +279,16 @@ def forward(q, k, v, causal=False, scale=None, out=None, lse=None, stream=None):
         lse = torch.empty((B, H, Sq), dtype=torch.float32, device=dev)
     _expect("out", out, (B, Sq, H, D), q.dtype, dev)
     _expect_lse(lse, B, H, Sq, dev)
-    p = FwdParams(_view(q), _view(k), _view(v), _view(out), lse.data_ptr(),
-                  B, H, Sq, Sk, D, float(scale), int(bool(causal)), dt)
+    views = (_view(q), _view(k), _view(v), _view(out))  # refuses non-CUDA tensors first
+    if workspace is None and split_ranks >= 0:
+        workspace = fwd_workspace_for(B, H, Sq, Sk, D, causal, dev, split_ranks)
+    if workspace is not None:
+        if workspace.device != dev or workspace.dtype != torch.uint8 or not workspace.is_contiguous():
+            raise ValueError("workspace: expected a contiguous uint8 tensor on q's device")
+    p = FwdParams(*views, lse.data_ptr(),
+                  B, H, Sq, Sk, D, float(scale), int(bool(causal)), dt,
+                  workspace.data_ptr() if workspace is not None else None,
+                  workspace.numel() if workspace is not None else 0, int(split_ranks))
     with torch.cuda.device(dev):
         st = fa_fwd_ex(p, _stream(stream))
     if st != FA_OK:

@@ -46,6 +46,7 @@ class HostAttentionPipeline:
                 "q": mk(), "k": mk(), "v": mk(), "do": mk(), "o": mk(), "dq": mk(), "dk": mk(), "dv": mk(),
                 "lse": torch.empty((B, H, S), dtype=torch.float32, device=self.device),
                 "ws": fa.workspace_for(B, H, S, D, self.device, Sk=S, deterministic=self.deterministic),
+                "fws": fa.fwd_workspace_for(B, H, S, S, D, causal, self.device),
                 # compute done with this set's inputs / forward outputs ready / results copied out
                 "computed": torch.cuda.Event(), "fwd_done": torch.cuda.Event(), "copied_out": torch.cuda.Event(),
                 "copied_in": torch.cuda.Event(), "used": False,
@@ -81,7 +82,8 @@ class HostAttentionPipeline:
             if st["used"]:
                 self.s_comp.wait_event(st["copied_out"])    # the previous results left the device
             fa.forward(st["q"], st["k"], st["v"], causal=self.causal, scale=self.scale, out=st["o"],
-                       lse=st["lse"], stream=self.s_comp)
+                       lse=st["lse"], stream=self.s_comp, workspace=st["fws"],
+                       split_ranks=0 if st["fws"] is not None else -1)
             st["fwd_done"].record(self.s_comp)
             fa.backward(st["q"], st["k"], st["v"], st["o"], st["lse"], st["do"], causal=self.causal,
                         scale=self.scale, dq=st["dq"], dk=st["dk"], dv=st["dv"], workspace=st["ws"],

@@ -109,6 +109,29 @@ typedef struct {
   float scale;
   int causal; /* 0 or 1 */
   int dtype;  /* fa_dtype */
+  /* Optional key-range split (all three zero: off). With a workspace of at
+     least fa_fwd_workspace_size_ex(B, H, Sq, Sk, D, causal, split_ranks, NULL)
+     bytes (256-byte aligned, used by no other call at the same time, need not
+     be initialised) the heaviest 256-row query blocks may each run as two
+     CTAs, one per half of the key blocks, whose partial results are merged
+     exactly (the online-softmax rescaling of [P4] §3.1 applied between the
+     two halves); this shortens the longest CTA and fills the SMs when
+     B * H * ceil(Sq / 256) is small ([P4] §3.2: too few blocks for the SMs).
+     O and lse stay the exact attention; the rounding order differs from the
+     unsplit CTAs in the last bits. split_ranks: 0 = the library chooses
+     (a list-scheduling estimate of the CTAs over the current device's SMs,
+     kept if it predicts a grid more than 5% shorter; never splits at four
+     waves or more), k > 0 = split the first min(k,
+     ceil(Sq / 256)) query-block ranks (ranks count 256-row blocks from the
+     last one when causal, the heaviest first; from the first otherwise),
+     -1 = never. Splits apply only when ceil(Sq / 256) <= 64. The CTAs then
+     start longest first (whole ranks and halves sorted by their estimated
+     length). A NULL workspace runs unsplit; a non-NULL workspace that is
+     too small for the split chosen is FA_ERR_WORKSPACE, a misaligned one
+     FA_ERR_MISALIGNED. */
+  void* workspace;
+  size_t workspace_bytes;
+  int split_ranks;
 } fa_fwd_params;
 
 typedef struct {
@@ -132,13 +155,24 @@ typedef struct {
 
 /* Forward ([P1] "性能引擎"; [P2] items 1-2; [P4] §3.1, §3.2).
    Reads q [B,Sq,H,D], k and v [B,Sk,H,D]; writes o [B,Sq,H,D] (rounded once,
-   to nearest even, to `dtype`) and lse [B,H,Sq] fp32. Dense tensors. */
+   to nearest even, to `dtype`) and lse [B,H,Sq] fp32. Dense tensors; no
+   workspace, so no key-range split (fa_fwd_ex has it). */
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
            int B, int H, int Sq, int Sk, int D, float scale, int causal,
            int dtype, fa_stream_t stream);
 
-/* Forward on strided views (packed qkv and the like). Same semantics. */
+/* Forward on strided views (packed qkv and the like), with the optional
+   key-range split. Same semantics. */
 int fa_fwd_ex(const fa_fwd_params* p, fa_stream_t stream);
+
+/* Workspace bytes fa_fwd_ex needs for the split that `split_ranks` selects
+   (see fa_fwd_params) on the current device; 0 when that is no split or the
+   arguments are invalid. If n_split is not NULL it receives the number of
+   split query-block ranks (0: none). Host only; launches nothing. */
+size_t fa_fwd_workspace_size_ex(int B, int H, int Sq, int Sk, int D, int causal, int split_ranks, int* n_split);
+
+/* fa_fwd_workspace_size_ex with split_ranks = 0 (the library's choice). */
+size_t fa_fwd_workspace_size(int B, int H, int Sq, int Sk, int D, int causal);
 
 /* e4m3 forward: the parameters of fa_fwd_fp8_ex. */
 typedef struct {

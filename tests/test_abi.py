@@ -151,6 +151,37 @@ def test_strided_views_checked(fa_lib):
     assert fa_lib.fa_bwd_ex(None, None) == -1
 
 
+def test_fwd_workspace_sizes(fa_lib):
+    """Forced key-range splits: tickets (8 B per split (b, h, rank)), then per
+    split CTA 256 rows of (m, l) and of fp32 O at the kernel width, each
+    section 256-byte aligned. No device is needed for a forced split."""
+    import ctypes
+    ns = ctypes.c_int(-1)
+    n = fa_lib.fa_fwd_workspace_size_ex(2, 3, 1000, 1000, 128, 1, 2, ctypes.byref(ns))
+    pairs, ctas = 2 * 3 * 2, 2 * 2 * 3 * 2
+    off_o = 256 + (ctas * 256 * 8 + 255) // 256 * 256
+    assert ns.value == 2 and n == off_o + ctas * 256 * 128 * 4 and pairs * 8 <= 256
+    # split_ranks above the number of 256-row ranks is capped (1000 rows: 4
+    # ranks); D = 40 runs the 64-wide kernel
+    n = fa_lib.fa_fwd_workspace_size_ex(2, 3, 1000, 1000, 40, 0, 9, ctypes.byref(ns))
+    ctas = 2 * 2 * 3 * 4
+    assert ns.value == 4 and n == 256 + (ctas * 256 * 8 + 255) // 256 * 256 + ctas * 256 * 64 * 4
+    assert fa_lib.fa_fwd_workspace_size_ex(2, 3, 1000, 1000, 64, 0, -1, ctypes.byref(ns)) == 0 and ns.value == 0
+    assert fa_lib.fa_fwd_workspace_size_ex(0, 3, 1000, 1000, 64, 0, 2, None) == 0
+    # no split past 64 ranks of 256 rows
+    assert fa_lib.fa_fwd_workspace_size_ex(1, 1, 64 * 256, 64 * 256, 64, 0, 2, ctypes.byref(ns)) > 0 and ns.value == 2
+    assert fa_lib.fa_fwd_workspace_size_ex(1, 1, 64 * 256 + 1, 64 * 256, 64, 0, 2, ctypes.byref(ns)) == 0
+    assert ns.value == 0
+    assert fa_lib.fa_fwd_workspace_size_ex(1, 1, 10, 10, 72, 0, 2, None) > 0    # D <= 128: the 128-wide kernel
+    assert fa_lib.fa_fwd_workspace_size_ex(1, 1, 10, 10, 144, 0, 2, None) == 0  # unsupported head_dim
+
+
+def test_fwd_workspace_alignment_checked(fa_lib):
+    t = fa.FaTensor(A, 512 * 12 * 64, 12 * 64, 64)
+    p = fa.FwdParams(t, t, t, t, A, 2, 12, 512, 512, 64, 0.125, 0, fa.FA_FP16, A + 16, 1 << 20, 1)
+    assert fa.fa_fwd_ex(p) == -3                 # workspace must be 256-byte aligned
+
+
 def test_bwd_ex_deterministic_flag_checked(fa_lib):
     t = fa.FaTensor(A, 512 * 12 * 64, 12 * 64, 64)
     ws = fa.fa_bwd_workspace_size_ex(2, 12, 512, 512, 64, 1)

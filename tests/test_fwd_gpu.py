@@ -89,3 +89,27 @@ def test_fwd_workloads_sampled(name):
         for h in range(w.H):
             o_ref, lse_ref = oracle.attention_forward_rows(qn, kn, vn, w.scale, causal, 0, h, rows)
             check_o_lse(o[0, rows, h], lse[0, h, rows], o_ref, lse_ref, w.dtype, f"{name} h{h} causal={causal}")
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+def test_fwd_masked_keys_weigh_zero(D, dtype):
+    """Causal: keys past a row's diagonal must get P exactly 0, not a tiny
+    weight. V on keys >= T is set to the largest power of two of the format
+    (2^127 in bf16, 2^15 in fp16): rows below T, which never see those keys,
+    must match the oracle and be bit-identical to a run with those V rows 0.
+    T = 448 cuts through the diagonal block of the second 256-row query
+    block, so element-wise masking is exercised."""
+    S, T = 512, 448
+    c = random_case(1, 2, S, S, D, dtype, 31 + D)
+    big = 2.0 ** 127 if dtype == torch.bfloat16 else 2.0 ** 15
+    v_big, v_zero = c["v"].clone(), c["v"].clone()
+    v_big[:, T:] = big
+    v_zero[:, T:] = 0
+    q, k = c["q"].cuda(), c["k"].cuda()
+    o_big, lse_big = run_fwd(q, k, v_big.cuda(), True)
+    o_zero, lse_zero = run_fwd(q, k, v_zero.cuda(), True)
+    assert torch.equal(o_big[:, :T], o_zero[:, :T]), "masked keys leaked into O"
+    assert torch.equal(lse_big, lse_zero)
+    o_ref, lse_ref = oracle.attention_forward(np64(c["q"]), np64(c["k"]), np64(v_big), D ** -0.5, True)
+    check_o_lse(np64(o_big[:, :T]), np64(lse_big), o_ref[:, :T], lse_ref, dtype, f"D{D} {dtype} huge masked V")
