@@ -231,7 +231,7 @@ double split_makespan(const int* c0, const int* c1, const SplitPlan& p, int HB, 
 
 // The plan for split_ranks (see fa_fwd_params): -1 none, k > 0 min(k, ranks),
 // 0 the estimate's best (kept only if it beats the unsplit grid by more than
-// 5%). No split past kMaxSplitRanks ranks. Automatic plans are cached per
+// 8%). No split past kMaxSplitRanks ranks. Automatic plans are cached per
 // shape.
 SplitPlan plan_split(int B, int H, int Sq, int Sk, int Dk, int causal, int split_ranks) {
   const int nq = (Sq + 255) / 256;
@@ -274,7 +274,7 @@ SplitPlan plan_split(int B, int H, int Sq, int Sk, int Dk, int causal, int split
       best = p;
     }
   }
-  if (best_t > 0.95 * base) best = none;
+  if (best_t > 0.92 * base) best = none;
   std::lock_guard<std::mutex> g(mu);
   cache[cache_next] = Entry{B, H, Sq, Sk, Dk, causal, sms, best};
   cache_next = (cache_next + 1) % 32;

@@ -312,9 +312,13 @@ __global__ void __launch_bounds__(448, 1)
   const float* s_dvec = reinterpret_cast<const float*>(smem + L::OFF_DVEC);
   constexpr int kLoaderWarp = 12, kMmaWarp = 13;
 
+  // Causal: key-block-major, the first key blocks (the most query blocks)
+  // first. Without a mask every CTA has the same length and the grid is
+  // head-major: the CTAs running at one time then share a few heads' Q, dO
+  // and dQ accumulator, which stay in L2.
   const int hb_count = a.H * a.B;
-  const int kvb = blockIdx.x / hb_count;  // causal: the first key blocks see the most queries
-  const int hb = blockIdx.x % hb_count;
+  const int kvb = a.causal ? static_cast<int>(blockIdx.x) / hb_count : static_cast<int>(blockIdx.x) % a.nkb;
+  const int hb = a.causal ? static_cast<int>(blockIdx.x) % hb_count : static_cast<int>(blockIdx.x) / a.nkb;
   const int h = hb % a.H;
   const int b = hb / a.H;
   const int n0 = kvb * L::BN;

@@ -308,9 +308,13 @@ __global__ void __launch_bounds__(576, 1)
   // FwdArgs::order, longest first: a whole rank, or one half of a split rank
   // (half 0: key blocks [0, hs), half 1: [hs, n), hs = ceil(n / 2) of the
   // block's longer tile).
+  // Without a mask and unsplit, every CTA has the same length and the grid
+  // is head-major instead: the CTAs running at one time then share a few
+  // heads' K and V, which stay in L2.
   const int hb_count = a.H * a.B;
-  const int unit = blockIdx.x / hb_count;
-  const int hb = blockIdx.x % hb_count;
+  const bool head_major = !a.causal && a.n_split == 0;
+  const int unit = head_major ? static_cast<int>(blockIdx.x) % a.n_qblocks : blockIdx.x / hb_count;
+  const int hb = head_major ? static_cast<int>(blockIdx.x) / a.n_qblocks : blockIdx.x % hb_count;
   int rank = unit, half = 0;
   bool split = false;
   if (a.n_split > 0) {

@@ -120,7 +120,7 @@ typedef struct {
      O and lse stay the exact attention; the rounding order differs from the
      unsplit CTAs in the last bits. split_ranks: 0 = the library chooses
      (a list-scheduling estimate of the CTAs over the current device's SMs,
-     kept if it predicts a grid more than 5% shorter; never splits at four
+     kept if it predicts a grid more than 8% shorter; never splits at four
      waves or more), k > 0 = split the first min(k,
      ceil(Sq / 256)) query-block ranks (ranks count 256-row blocks from the
      last one when causal, the heaviest first; from the first otherwise),
