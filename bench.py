@@ -372,7 +372,7 @@ def run_ours(args, w, causal):
     peak_tf = peaks.get("bf16_tflops_sustained" if sustained else "bf16_tflops")
     # Dominant call of a step: the one with the larger share of device time.
     if t_bwd >= t_fwd:
-        dom, dom_flops, dom_t = "fa_bwd (fa_bwd_pre + fa_bwd_main + fa_bwd_dq)", fb, t_bwd_max / args.steps
+        dom, dom_flops, dom_t = "fa_bwd (fa_bwd_pre + fa_bwd_main + dQ convert)", fb, t_bwd_max / args.steps
     else:
         dom, dom_flops, dom_t = "fa_fwd_kernel", ff, t_fwd_max / args.steps
     achieved = dom_flops / dom_t / 1e12
