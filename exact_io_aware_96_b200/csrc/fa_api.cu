@@ -484,7 +484,7 @@ int noalloc_scratch(void** out) {
 
 extern "C" {
 
-int fa_version(void) { return 200; }
+int fa_version(void) { return 300; }
 
 const char* fa_strerror(int s) {
   switch (s) {
