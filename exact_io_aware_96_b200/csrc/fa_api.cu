@@ -233,7 +233,7 @@ double split_makespan(const int* c0, const int* c1, const SplitPlan& p, int HB, 
 // 0 the estimate's best (kept only if it beats the unsplit grid by more than
 // 8%). No split past kMaxSplitRanks ranks. Automatic plans are cached per
 // shape.
-SplitPlan plan_split(int B, int H, int Sq, int Sk, int Dk, int causal, int split_ranks) {
+SplitPlan plan_split(int B, int H, int Sq, int Sk, int Dk, int causal, int split_ranks, int sms) {
   const int nq = (Sq + 255) / 256;
   SplitPlan none;
   if (split_ranks < 0 || nq > fa::FwdArgs::kMaxSplitRanks) return none;
@@ -245,7 +245,6 @@ SplitPlan plan_split(int B, int H, int Sq, int Sk, int Dk, int causal, int split
   }
   const double merge = split_merge_cost(Dk);
   if (split_ranks > 0) return split_order(c0.data(), c1.data(), nq, std::min(split_ranks, nq), merge);
-  const int sms = sm_count();
   const int64_t HB = int64_t(B) * H;
   if (sms <= 0 || HB * nq >= 4 * int64_t(sms)) return none;
   struct Entry {
@@ -316,7 +315,7 @@ int launch_fwd(const fa_fwd_params* p, cudaStream_t stream) {
   a.n_qblocks = (p->Sq + 255) / 256;
   a.d = p->D;
   if (p->workspace != nullptr) {
-    const SplitPlan plan = plan_split(p->B, p->H, p->Sq, p->Sk, D, p->causal, p->split_ranks);
+    const SplitPlan plan = plan_split(p->B, p->H, p->Sq, p->Sk, D, p->causal, p->split_ranks, sm_count());
     const int ns = plan.ns;
     const SplitLayout sl = split_layout(p->B, p->H, ns, D);
     if (ns > 0) {
@@ -589,9 +588,24 @@ size_t fa_fwd_workspace_size_ex(int B, int H, int Sq, int Sk, int D, int causal,
   if (n_split != nullptr) *n_split = 0;
   if (check_common(B, H, Sq, Sk, D, 1.f, causal, FA_BF16) != FA_OK) return 0;
   const int Dk = D <= 64 ? 64 : 128;
-  const int ns = plan_split(B, H, Sq, Sk, Dk, causal, split_ranks).ns;
+  const int ns = plan_split(B, H, Sq, Sk, Dk, causal, split_ranks, sm_count()).ns;
   if (n_split != nullptr) *n_split = ns;
   return size_t(split_layout(B, H, ns, Dk).bytes);
+}
+
+int fa_fwd_split_plan(int B, int H, int Sq, int Sk, int D, int causal, int split_ranks, int sms, int* n_split,
+                      unsigned char* order, int order_capacity) {
+  if (n_split != nullptr) *n_split = 0;
+  int st = check_common(B, H, Sq, Sk, D, 1.f, causal, FA_BF16);
+  if (st != FA_OK) return st;
+  if (sms < 0 || order_capacity < 0 || (order == nullptr && order_capacity > 0)) return FA_ERR_INVALID_ARG;
+  if (sms == 0 && (sms = sm_count()) <= 0) return FA_ERR_CUDA;
+  const SplitPlan plan = plan_split(B, H, Sq, Sk, D <= 64 ? 64 : 128, causal, split_ranks, sms);
+  if (n_split != nullptr) *n_split = plan.ns;
+  if (plan.ns == 0) return 0;
+  if (order_capacity < plan.units) return FA_ERR_INVALID_ARG;
+  std::memcpy(order, plan.order, size_t(plan.units));
+  return plan.units;
 }
 
 size_t fa_fwd_workspace_size(int B, int H, int Sq, int Sk, int D, int causal) {

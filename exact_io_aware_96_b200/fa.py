@@ -31,7 +31,7 @@ STATUS = {
 }
 FA_NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 EXPORTED = ("fa_fwd", "fa_fwd_ex", "fa_fwd_fp8", "fa_fwd_fp8_ex", "fa_bwd", "fa_bwd_ex", "fa_bwd_noalloc",
-            "fa_fwd_workspace_size", "fa_fwd_workspace_size_ex",
+            "fa_fwd_workspace_size", "fa_fwd_workspace_size_ex", "fa_fwd_split_plan",
             "fa_bwd_workspace_size", "fa_bwd_workspace_size_ex", "fa_selftest_wait_timeout",
             "fa_last_device_status", "fa_strerror", "fa_version")
 
@@ -114,6 +114,8 @@ def lib():
         L.fa_fwd_workspace_size.restype = sz
         L.fa_fwd_workspace_size_ex.argtypes = [i, i, i, i, i, i, i, ctypes.POINTER(ctypes.c_int)]
         L.fa_fwd_workspace_size_ex.restype = sz
+        L.fa_fwd_split_plan.argtypes = [i, i, i, i, i, i, i, i, ctypes.POINTER(ctypes.c_int), ctypes.c_void_p, i]
+        L.fa_fwd_split_plan.restype = i
         L.fa_bwd_workspace_size.argtypes = [i, i, i, i]
         L.fa_bwd_workspace_size.restype = sz
         L.fa_bwd_workspace_size_ex.argtypes = [i, i, i, i, i, i]
@@ -251,6 +253,18 @@ def fwd_workspace_size(B, H, Sq, Sk, D, causal, split_ranks=0, device=None):
     with torch.cuda.device(device if device is not None else torch.cuda.current_device()):
         n = lib().fa_fwd_workspace_size_ex(B, H, Sq, Sk, D, int(bool(causal)), int(split_ranks), ctypes.byref(ns))
     return int(n), ns.value
+
+
+def fwd_split_plan(B, H, Sq, Sk, D, causal, split_ranks=0, sms=0):
+    """(n_split, [(rank, kind), ...]) of the forward's key-range split for
+    `sms` SMs (0: the current device); kind 0 whole rank, 1/2 its key halves."""
+    ns = ctypes.c_int(0)
+    buf = (ctypes.c_ubyte * 256)()
+    n = lib().fa_fwd_split_plan(B, H, Sq, Sk, D, int(bool(causal)), int(split_ranks), int(sms), ctypes.byref(ns),
+                                buf, 256)
+    if n < 0:
+        raise FaError(n, "fa_fwd_split_plan")
+    return ns.value, [(buf[i] // 3, buf[i] % 3) for i in range(n)]
 
 
 def fwd_workspace_for(B, H, Sq, Sk, D, causal, device, split_ranks=0):

@@ -174,6 +174,20 @@ size_t fa_fwd_workspace_size_ex(int B, int H, int Sq, int Sk, int D, int causal,
 /* fa_fwd_workspace_size_ex with split_ranks = 0 (the library's choice). */
 size_t fa_fwd_workspace_size(int B, int H, int Sq, int Sk, int D, int causal);
 
+/* The key-range split plan, for inspection (host only; launches nothing).
+   Plans for `sms` SMs (0: the current device's count). *n_split receives
+   the number of split query-block ranks. If it is 0 the grid is rank-major
+   (head-major without a mask) and 0 is returned. Otherwise `order`
+   receives the grid's units, longest first, one byte each: rank * 3 + kind
+   (kind 0 = the whole rank, 1 = its first key half, 2 = its second). Ranks
+   count 256-row query blocks from the last one when causal, from the first
+   otherwise. Each unit is B * H CTAs. The return value is the number of
+   units (ceil(Sq / 256) + n_split). Errors: as fa_fwd for the sizes;
+   FA_ERR_INVALID_ARG if sms < 0 or `order_capacity` is too small;
+   FA_ERR_CUDA if sms is 0 and no device can be queried. */
+int fa_fwd_split_plan(int B, int H, int Sq, int Sk, int D, int causal, int split_ranks, int sms, int* n_split,
+                      unsigned char* order, int order_capacity);
+
 /* e4m3 forward: the parameters of fa_fwd_fp8_ex. */
 typedef struct {
   fa_tensor q, k, v; /* read, E4M3 bytes; strides in elements (= bytes) */

@@ -13,7 +13,7 @@ import oracle
 import oracle.fp8
 from exact_io_aware_96_b200 import build, fa
 from exact_io_aware_96_b200.inputs import quantize_e4m3, random_case
-from tests.parity import check_fp8_o_lse, full_check, np64, rel_l2
+from tests.parity import check_fp8_o_lse, check_o_lse, full_check, np64, rel_l2
 
 pytestmark = pytest.mark.gpu
 
@@ -81,3 +81,20 @@ def test_check_build_e4m3(check_lib, Sq, Sk, causal):
         rows = np.arange(Sq)
         check_fp8_o_lse(np64(o)[0, :, h], np64(lse)[0, h], dq8["q"], dq8["k"], dq8["v"], 128 ** -0.5, causal,
                         torch.bfloat16, 0, h, rows, f"check build e4m3 h{h}")
+
+
+@pytest.mark.parametrize("Sq,Sk,D,causal", [(1000, 1000, 128, True), (700, 129, 64, True), (513, 300, 96, False),
+                                            (300, 1, 64, False)])
+def test_check_build_split_forward(check_lib, Sq, Sk, D, causal):
+    """The forward with every query-block rank split by key range (the
+    workspace slots, the tickets and the unit order are all checked sites)."""
+    c = random_case(2, 3, Sq, Sk, D, torch.bfloat16, 950 + Sq + D)
+    q, k, v = (c[n].cuda() for n in ("q", "k", "v"))
+    n, ns = fa.fwd_workspace_size(2, 3, Sq, Sk, D, causal, 64)
+    assert ns == (Sq + 255) // 256
+    ws = torch.full((n,), 255, dtype=torch.uint8, device="cuda")
+    o, lse = fa.forward(q, k, v, causal=causal, split_ranks=64, workspace=ws)
+    torch.cuda.synchronize()
+    _status_clear(f"split forward Sq{Sq} Sk{Sk} D{D}")
+    o_ref, lse_ref = oracle.attention_forward(np64(c["q"]), np64(c["k"]), np64(c["v"]), D ** -0.5, causal)
+    check_o_lse(np64(o), np64(lse), o_ref, lse_ref, torch.bfloat16, f"check build split Sq{Sq} Sk{Sk} D{D}")
