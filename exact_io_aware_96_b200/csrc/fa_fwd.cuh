@@ -440,10 +440,17 @@ __global__ void __launch_bounds__(576, 1)
         checked(buf + 128 <= OBASE && st < S && t < 2, 103);
         const uint64_t qd = desc_sw128(sQ + t * L::TILE, 16, 1024);
         const uint64_t kd = desc_sw128(sK + st * L::TILE, 16, 1024);
+        // 32 bytes of the head dim per instruction, four instructions per
+        // 128-byte column block, issued under one elect.
 #pragma unroll
-        for (int kk = 0; kk < L::RB / 32; ++kk) {  // 32 bytes of the head dim per instruction
-          const uint32_t o = (kk >> 2) * L::BLK + (kk & 3) * 32;
-          mma_ss_w(tmem + buf, desc_add(qd, o), desc_add(kd, o), idS, kk > 0);
+        for (int kb = 0; kb < L::KB; ++kb) {
+          uint64_t ad[4], bd[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            ad[u] = desc_add(qd, kb * L::BLK + u * 32);
+            bd[u] = desc_add(kd, kb * L::BLK + u * 32);
+          }
+          mma_ss_x4(tmem + buf, ad, bd, idS, kb > 0);
         }
       };
       // O_t += P_t V with P_t over the S buffer at `buf`.
@@ -453,9 +460,16 @@ __global__ void __launch_bounds__(576, 1)
         // Keys 16kk .. 16kk + 15: P of half kk >> 2 at columns buf + 64(kk >> 2)
         // + 8(kk & 3) (8 columns per 16 keys); V advances 16 rows of 128 bytes.
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts_w(tmem + OBASE + t * D, tmem + buf + 64 * (kk >> 2) + (kk & 3) * 8, desc_add(vd, kk * 2048), idO,
-                   (acc || kk > 0) ? 1u : 0u);
+        for (int h = 0; h < 2; ++h) {  // the two halves of P, four instructions each under one elect
+          uint32_t pa[4];
+          uint64_t vb[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            pa[u] = tmem + buf + 64 * h + u * 8;
+            vb[u] = desc_add(vd, (4 * h + u) * 2048);
+          }
+          mma_ts_x4(tmem + OBASE + t * D, pa, vb, idO, (acc || h > 0) ? 1u : 0u);
+        }
       };
       bool ok = wait(q_full, 0, -1);
       if constexpr (kRot3) {
