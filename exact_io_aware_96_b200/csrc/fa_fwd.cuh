@@ -649,7 +649,9 @@ __global__ void __launch_bounds__(576, 1)
         continue;
       }
       if (rescale) {
-        // Rescale this warp's 32 rows of this half's D/2 columns of O_t.
+        // Rescale this warp's 32 rows of this half's D/2 columns of O_t. The
+        // fence orders the TMEM loads after the wait above.
+        tc_fence_after();
 #pragma unroll 1
         for (int q = 0; q < D / 64; ++q) {
           uint32_t ov[32];

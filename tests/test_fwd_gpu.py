@@ -53,6 +53,16 @@ def test_fwd_wide_scores():
     _fwd_case(1, 2, 1000, 1000, 128, torch.bfloat16, True, seed=12, qk_std=4.0)
 
 
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("qk_std", [3.0, 6.0])
+@pytest.mark.parametrize("S", [300, 1000, 1500])
+def test_fwd_wide_scores_d64(causal, qk_std, S):
+    """D = 64 rescales O_t while later S products are already in flight (three
+    rotating S buffers): the running max must be raised on the last and the
+    middle blocks of a tile alike."""
+    _fwd_case(2, 2, S, S, 64, torch.float16, causal, seed=int(13 * qk_std) + S, qk_std=qk_std)
+
+
 def test_fwd_repeatable():
     c = random_case(1, 4, 777, 777, 128, torch.bfloat16, 3)
     q, k, v = c["q"].cuda(), c["k"].cuda(), c["v"].cuda()
